@@ -1,0 +1,462 @@
+#!/usr/bin/env python
+"""Benchmark of one hybrid compressed attention layer on B200.
+
+Headline: CSA prefill of a 32K-token sequence (bf16, 64 query heads sharing one
+128-d K/V, r = 4 with windows of 8 at stride 4, indexer dim 128, flat top-512,
+128-token window).  One step = S1 compression of the whole sequence + S2 flat
+indexer and top-k for every query + S3/S4 attention for every query.
+value = tokens/s over all ranks (replicas: each rank runs the whole layer).
+Also reported: the decode step of 64 sequences x 128K context (CSA flat top-512
++ HCA dense), per-stage times, the roofline of the dominant kernel, an
+end-to-end figure through host buffers, SM clocks during the timed region, and
+the fp64 CPU oracle timed on a bounded sample.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import configs as C  # noqa: E402
+from workloads import make, rng  # noqa: E402
+
+METRIC = "prefill tok/s & decode tok/s per hybrid layer at 1 B200; % of HBM/TC roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU oracle sample")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: d[k] for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- distributed plumbing
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- workload
+
+
+def prefill_inputs(w, device):
+    ly = w.layer("csa")
+    raw, qs = make.make_raw(w, device), make.make_queries(w, device)
+    make.plant_prefill(w, ly, raw, qs, device)
+    bias = make.make_bias(w, ly, device)
+    return raw, qs, bias
+
+
+def attention_flops(w, ly, q_pos: np.ndarray, n_c: int) -> float:
+    """4*H*D per (query, key): keys = min(k, visible entries) + window length (CSA),
+    or all visible entries + window length (HCA)."""
+    t = q_pos.astype(np.int64)
+    vis = np.minimum((t + 1) // ly.r, n_c)
+    comp = np.minimum(vis, ly.k) if ly.kind == "csa" else vis
+    win = np.minimum(w.W, t + 1)
+    return 4.0 * w.H * w.D * float((comp + win).sum())
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "sparse_attention_hyb_b200", "csrc", "*"))):
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was
+    taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d or d.get("source_hash") != source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class PrefillStep:
+    """All buffers of one CSA prefill layer, preallocated; run() enqueues the three calls."""
+
+    def __init__(self, S, w, raw, qs, bias):
+        self.S, self.w, self.ly = S, w, w.layer("csa")
+        self.raw, self.qs, self.bias = raw, qs, bias
+        ly, dev = self.ly, raw["xk"].device
+        L = raw["xk"].shape[1]
+        self.n_c = L // ly.r
+        self.kc = torch.empty(1, self.n_c, w.D, dtype=raw["xk"].dtype, device=dev)
+        self.vc = torch.empty_like(self.kc)
+        self.ic = torch.empty(1, self.n_c, w.dI, dtype=raw["xk"].dtype, device=dev)
+        self.idx = torch.empty(1, w.T, ly.k, dtype=torch.int32, device=dev)
+        self.o = torch.empty_like(qs["q"])
+        self.lse = torch.empty(1, w.T, w.H, dtype=torch.float32, device=dev)
+        A = S.abi
+        nb = A.hyb_index_topk_workspace_size(A.HYB_DTYPE_BF16, 1, w.T, self.n_c, w.dI, ly.k, A.HYB_INDEX_FLAT)
+        self.ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+        self.scale = 1.0 / math.sqrt(w.D)
+
+    def run(self, ev=None):
+        A, ly, raw, qs = self.S.abi, self.ly, self.raw, self.qs
+        if ev:
+            ev[0].record()
+        A.hyb_compress(raw["xk"], raw["xv"], raw["xi"], raw["z"], self.bias, ly.r, ly.overlap, 0, self.n_c,
+                       self.kc, self.vc, self.ic)
+        if ev:
+            ev[1].record()
+        A.hyb_index_topk(qs["qi"], qs["q_pos"], self.ic, self.n_c, ly.r, ly.k, A.HYB_INDEX_FLAT, None, 0, 0, 0,
+                         self.idx, self.ws)
+        if ev:
+            ev[2].record()
+        A.hyb_attn_fwd(qs["q"], qs["q_pos"], self.kc, self.vc, self.n_c, ly.r, self.idx, ly.k, raw["xk"],
+                       raw["xv"], self.w.W, self.scale, self.o, self.lse, A.HYB_ATTN_PREFILL, None)
+        if ev:
+            ev[3].record()
+
+
+def bench_prefill(S, w, steps, warmup, world, flush):
+    raw, qs, bias = prefill_inputs(w, "cuda")
+    st = PrefillStep(S, w, raw, qs, bias)
+    for _ in range(warmup):
+        st.run()
+    torch.cuda.synchronize()
+    if S.abi.hyb_get_device_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    n0 = S.abi.hyb_kernel_launches()
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()                      # evict L2 between timed steps (outside the events)
+        st.run(evs[i])
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = S.abi.hyb_kernel_launches() - n0
+    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(steps)])
+    step_ms = float(stage.sum(axis=1).mean())
+    flops = attention_flops(w, st.ly, qs["q_pos"][0].cpu().numpy(), st.n_c)
+    return st, {"step_ms": step_ms, "stage_ms": stage.mean(axis=0).tolist(), "launches": launches,
+                "attn_flops": flops}
+
+
+def bench_e2e(S, st, steps):
+    """Same step through host buffers: pinned H2D of every input, the three calls,
+    D2H of o and lse, all inside the timed region."""
+    names = ["xk", "xv", "xi", "z"]
+    host_raw = {k: st.raw[k].cpu().pin_memory() for k in names}
+    host_q = {k: st.qs[k].cpu().pin_memory() for k in ("q", "qi", "q_pos")}
+    host_b = st.bias.cpu().pin_memory()
+    out_o = torch.empty(st.o.shape, dtype=st.o.dtype, pin_memory=True)
+    out_l = torch.empty(st.lse.shape, dtype=st.lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in list(host_raw.values()) + list(host_q.values())) \
+        + host_b.numel() * 4
+    d2h = out_o.numel() * out_o.element_size() + out_l.numel() * 4
+
+    def one():
+        for k in names:
+            st.raw[k].copy_(host_raw[k], non_blocking=True)
+        for k in host_q:
+            st.qs[k].copy_(host_q[k], non_blocking=True)
+        st.bias.copy_(host_b, non_blocking=True)
+        st.run()
+        out_o.copy_(st.o, non_blocking=True)
+        out_l.copy_(st.lse, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def bench_decode(S, steps, warmup, flush):
+    w = C.DECODE_BS64_128K
+    qs = make.make_queries(w, "cuda")
+    cache = make.make_decode_cache(w, "cuda")
+    make.plant_decode(w, w.layer("csa"), cache, qs, "cuda")
+    A = S.abi
+    csa, hca = w.layer("csa"), w.layer("hca")
+    nc_c, nc_h = w.L // csa.r, w.L // hca.r
+    idx = torch.empty(w.batch, 1, csa.k, dtype=torch.int32, device="cuda")
+    o = torch.empty_like(qs["q"])
+    o2 = torch.empty_like(qs["q"])
+    lse = torch.empty(w.batch, 1, w.H, dtype=torch.float32, device="cuda")
+    lse2 = torch.empty_like(lse)
+    wsi = torch.empty(max(256, A.hyb_index_topk_workspace_size(1, w.batch, 1, nc_c, w.dI, csa.k, 0)),
+                      dtype=torch.uint8, device="cuda")
+    wsa = torch.empty(max(256, A.hyb_attn_fwd_workspace_size(1, w.batch, 1, w.H, w.D, csa.k, nc_c, w.W, 1)),
+                      dtype=torch.uint8, device="cuda")
+    wsh = torch.empty(max(256, A.hyb_attn_fwd_workspace_size(1, w.batch, 1, w.H, w.D, 0, nc_h, w.W, 1)),
+                      dtype=torch.uint8, device="cuda")
+    scale = 1.0 / math.sqrt(w.D)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        A.hyb_index_topk(qs["qi"], qs["q_pos"], cache["ic"], nc_c, csa.r, csa.k, A.HYB_INDEX_FLAT, None, 0, 0, 0,
+                         idx, wsi)
+        A.hyb_attn_fwd(qs["q"], qs["q_pos"], cache["kc_csa"], cache["vc_csa"], nc_c, csa.r, idx, csa.k,
+                       cache["kw"], cache["vw"], w.W, scale, o, lse, A.HYB_ATTN_DECODE, wsa)
+        if ev:
+            ev[1].record()
+        A.hyb_attn_fwd(qs["q"], qs["q_pos"], cache["kc_hca"], cache["vc_hca"], nc_h, hca.r, None, 0,
+                       cache["kw"], cache["vw"], w.W, scale, o2, lse2, A.HYB_ATTN_DECODE, wsh)
+        if ev:
+            ev[2].record()
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    csa_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    hca_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    bytes_csa = w.batch * (nc_c * w.dI * 2 + (csa.k + w.W) * 2 * w.D * 2 + 2 * w.H * w.D * 2)
+    bytes_hca = w.batch * ((nc_h + w.W) * 2 * w.D * 2 + 2 * w.H * w.D * 2)
+    return {"workload": w.name, "tokens_per_s_csa_plus_hca": w.batch / ((csa_ms + hca_ms) / 1e3),
+            "tokens_per_s_csa": w.batch / (csa_ms / 1e3), "tokens_per_s_hca": w.batch / (hca_ms / 1e3),
+            "ms_csa": csa_ms, "ms_hca": hca_ms,
+            "hbm_gbs_csa": bytes_csa / (csa_ms / 1e3) / 1e9, "hbm_gbs_hca": bytes_hca / (hca_ms / 1e3) / 1e9,
+            "algorithmic_bytes_csa": bytes_csa, "algorithmic_bytes_hca": bytes_hca}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+
+def oracle_sample(w, seconds: float):
+    """Times the fp64 oracle on host cores: S1 over the whole sequence, then S2+S3
+    row by row until the budget is spent.  Returns (tokens/s, rows, seconds, cores)."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(1)
+    except ImportError:
+        limit = None
+    torch.set_num_threads(os.cpu_count() or 1)
+    ly = w.layer("csa")
+    raw = make.make_raw(w)
+    qi = make.normal_tensor(w.seed, "q_index", (w.batch, w.T, w.dI), w.i_scale, w.dtype)
+    qs = {"qi": qi, "q_pos": make.query_positions(w)}
+    make.plant_prefill(w, ly, raw, qs)
+    bias = make.make_bias(w, ly)
+    f64 = lambda t: t.float().double().numpy()
+    p = O.LayerParams("csa", ly.r, ly.overlap, w.W, 1.0 / math.sqrt(w.D), w.dtype, k=ly.k)
+    t0 = time.perf_counter()
+    kc, vc, ic = O.build_caches(p, f64(raw["xk"][0]), f64(raw["xv"][0]), f64(raw["xi"][0]), f64(raw["z"][0]),
+                                f64(bias))
+    t_s1 = time.perf_counter() - t0
+    xk, xv, qi64 = f64(raw["xk"][0]), f64(raw["xv"][0]), f64(qs["qi"][0])
+    order = torch.argsort(rng.raw_u64(w.seed, "cpu_rows", 0, w.T)).numpy()
+    done, t_rows = 0, 0.0
+    hd = w.H * w.D
+    while t_rows < seconds and done < w.T:
+        i = int(order[done])
+        q_row = make.to_storage(rng.normal(w.seed, "q", i * hd, hd) * w.x_scale, w.dtype).float().double()
+        t1 = time.perf_counter()
+        O.layer_row(p, q_row.view(w.H, w.D).numpy(), qi64[i], w.q_pos0 + i, kc, vc, ic, None, xk, xv, xk.shape[0])
+        t_rows += time.perf_counter() - t1
+        done += 1
+    if limit is not None:
+        limit.unregister() if hasattr(limit, "unregister") else None
+    per_row = t_rows / done + t_s1 / w.T
+    return 1.0 / per_row, done, t_rows + t_s1, 1
+
+
+# --------------------------------------------------------------------------- arms
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = C.PREFILL_32K
+    tok_s, rows, secs, cores = oracle_sample(w, max(2.0, args.cpu_seconds / max(1, args.steps)))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.T / tok_s,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "L": w.L, "T": w.T, "H": w.H, "D": w.D, "dI": w.dI, "r": 4, "k": 512,
+                   "W": w.W},
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"S1 over all {w.L} tokens + S2/S3 for {rows} seeded rows ({secs:.1f} s)"},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import sparse_attention_hyb_b200 as S
+    S.abi.lib()
+    w = C.PREFILL_32K
+    pk, pk_src = peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    clock = ClockSampler(local)
+    clock.start()
+    st, res = bench_prefill(S, w, args.steps, args.warmup, world, flush)
+    clocks = clock.stop()
+    step_ms = max_over_ranks(res["step_ms"], world)
+    value = world * w.T / (step_ms / 1e3)
+    attn_ms = res["stage_ms"][2]
+    achieved = res["attn_flops"] / (attn_ms / 1e3) / 1e12
+    peak = pk["bf16_tflops"]
+    traffic = measured_traffic("attention")
+    e2e_ms, h2d, d2h = bench_e2e(S, st, max(3, args.steps // 2))
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    decode = None if args.no_decode else bench_decode(S, args.steps, args.warmup, flush)
+    if S.abi.hyb_get_device_status() != 0:
+        raise RuntimeError("device status error after the benchmark")
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tok_s, rows, secs, cores = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"S1 over all {w.L} tokens + S2/S3 for {rows} seeded query rows ({secs:.1f} s, 1 thread)"}
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "L": w.L, "T": w.T, "H": w.H, "D": w.D, "dI": w.dI, "r": 4,
+                   "window_span": 8, "k": 512, "W": w.W, "parallelism": f"replicas{world}",
+                   "l2": "flushed (256 MiB write) between timed steps, outside the timed events"},
+        "stages_ms": {"compress": res["stage_ms"][0], "index_topk": res["stage_ms"][1],
+                      "attention": res["stage_ms"][2]},
+        "roofline": {"kernel": "attention (hyb_attn_fwd, prefill)", "bound": "tensor", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{pk_src} bf16 burst", "flops_per_launch": res["attn_flops"]},
+        "gpu_launches": res["launches"],
+        "e2e": {"value": world * w.T / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+        "decode": decode,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,178 @@
+/*
+ * hyb.h — C ABI of libhyb: the forward pass of one hybrid compressed attention
+ * layer (CSA: compressed + sparse; HCA: heavily compressed + dense) on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method is described on public pages only:
+ *  - "Hybrid Attention" explainer (process-cxr.github.io), section
+ *    "DeepSeek V4 中的定义": CSA compresses the KV cache along the sequence and
+ *    applies sparse attention; HCA compresses harder and attends densely.
+ *  - HCA article (daiw.net, "前代 · HCA：128 倍压缩后再做稠密注意力"), section
+ *    "怎么压" (How it is compressed) and the CSA/HCA table: softmax-weighted
+ *    pooling with a learnable positional bias, r = 128 without overlap (CSA:
+ *    r = 4, overlapping), shared-KV (MQA) attention, a 128-token sliding window.
+ *  - HISA write-up (my.qihongyi.cn, "DeepSeek速度狂飙4倍还不丢精度"), sections
+ *    01, 02 and 05, Fig. 2: flat top-k indexer; two-stage block/token indexer.
+ *  - trdm.cn news 749237, section 2.1: CSA = 4:1 compression + indexer top-k +
+ *    128-token window; HCA = 128:1 compression + dense attention.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    allocates nothing, keeps no pointer after returning and never
+ *    synchronises (except hyb_get_device_status).  Work is enqueued on
+ *    `stream` (a cudaStream_t; NULL = legacy default stream).
+ *  - Tensors are dense row-major with the batch dimension outermost; shapes
+ *    are given per argument.  `dtype` is HYB_DTYPE_F32 or HYB_DTYPE_BF16 and
+ *    applies to every non-fp32-typed tensor of the call (logits, bias and lse
+ *    are always fp32; positions and indices int32).
+ *  - Positions are absolute token positions (0-based).  Compressed entry j
+ *    covers raw tokens [(j-1)r, (j+1)r) (overlap = 1, clipped at 0) or
+ *    [jr, (j+1)r) (overlap = 0) and is visible to the query at position t iff
+ *    j < floor((t+1)/r) (its last token is at or before t).
+ *  - Return value: HYB_OK, or an error code from argument checks done on the
+ *    host before anything is launched (nothing is enqueued on error), or
+ *    HYB_ERR_CUDA when a launch failed.  Errors found by the kernels
+ *    themselves (an index out of range, a bounded wait that gave up) are
+ *    recorded in a per-device status word, read and cleared by
+ *    hyb_get_device_status.  No call traps, asserts or spins without bound.
+ *  - Calls are thread-safe and keep no state between calls other than the
+ *    per-device status word.
+ */
+#ifndef HYB_H_
+#define HYB_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hyb_stream_t; /* same type as cudaStream_t */
+
+enum {
+  HYB_OK = 0,
+  HYB_ERR_INVALID_ARG = 1,  /* null pointer, negative or inconsistent size    */
+  HYB_ERR_UNSUPPORTED = 2,  /* dtype, size or alignment outside what is built */
+  HYB_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required     */
+  HYB_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed           */
+  HYB_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up (status word)   */
+  HYB_ERR_DEVICE_CHECK = 6  /* device: an index or size check failed (status) */
+};
+
+enum { HYB_DTYPE_F32 = 0, HYB_DTYPE_BF16 = 1 };
+enum { HYB_INDEX_FLAT = 0, HYB_INDEX_HISA = 1 };
+enum { HYB_ATTN_PREFILL = 0, HYB_ATTN_DECODE = 1 };
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* hyb_status_string(int status);
+
+/* ABI version of this header (major*100 + minor). */
+int hyb_abi_version(void);
+
+/* Number of kernels this library has launched in this process (all devices),
+ * counted on the host at launch time: launch accounting for benchmarks. */
+unsigned long long hyb_kernel_launches(void);
+
+/*
+ * Reads the calling device's status word after synchronising `stream`, stores
+ * it in *status (HYB_OK when no kernel reported an error since the last read)
+ * and clears it.  Returns HYB_ERR_CUDA if the copy or synchronisation failed.
+ */
+int hyb_get_device_status(hyb_stream_t stream, int* status);
+
+/*
+ * S1 — sequence-axis compression (HCA article, section "怎么压"; CSA/HCA table;
+ * trdm.cn 2.1).  For every batch b and entry j in [j_begin, j_end):
+ *   w_i = softmax over the window of (logits[b, i] + bias[p]),
+ *   p = i - window_start(j) (position in the unclipped window),
+ *   kc[b, j] = sum_i w_i xk[b, i];  vc[b, j] = sum_i w_i xv[b, i];
+ *   ic[b, j] = sum_i w_i xi[b, i]  (when xi != NULL).
+ * The weights are computed in fp32 and the sums accumulated in fp32.
+ *   xk, xv  [batch, L, D]       xi [batch, L, dI] or NULL (then ic unused)
+ *   logits  [batch, L] fp32     bias [2r] (overlap = 1) or [r] (overlap = 0) fp32
+ *   kc, vc  [batch, nc_cap, D]  ic [batch, nc_cap, dI]
+ * Requires 0 <= j_begin <= j_end <= nc_cap, j_end * r <= L (whole windows
+ * only), r >= 1, window length (2r or r) <= 256, D and dI multiples of 4.
+ */
+int hyb_compress(int dtype, int batch, int L, int D, int dI,
+                 const void* xk, const void* xv, const void* xi,
+                 const float* logits, const float* bias, int r, int overlap,
+                 int j_begin, int j_end,
+                 void* kc, void* vc, void* ic, int nc_cap,
+                 hyb_stream_t stream);
+
+/*
+ * HISA stage-1 representatives (HISA write-up, section 02, stage 1: each block
+ * of `block` entries is summarised by one pooled vector; the mean is used).
+ * For blocks g in [g_begin, g_end): reps[b, g] = mean of ic[b, g*block ..
+ * (g+1)*block - 1], accumulated in fp32 and stored in `dtype`.
+ *   ic [batch, nc_cap, dI]   reps [batch, nb_cap, dI]
+ * Requires g_end * block <= nc_cap, g_end <= nb_cap, dI multiple of 4.
+ */
+int hyb_block_reps(int dtype, int batch, int dI, const void* ic, int nc_cap,
+                   int block, int g_begin, int g_end, void* reps, int nb_cap,
+                   hyb_stream_t stream);
+
+/*
+ * S2 — indexer and top-k selection (HISA write-up, sections 01 and 02; the
+ * output contract of section 05 step 3: k entry indices per query).
+ * Query (b, i) at position t = q_pos[b, i] sees entries j < V = min(floor((t+1)/r), nc);
+ * its score for entry j is qi[b, i] . ic[b, j] (fp32 accumulation).
+ *  mode HYB_INDEX_FLAT: keep the k best of the V entries.
+ *  mode HYB_INDEX_HISA: full visible blocks g < floor(V/block) are scored by
+ *    qi . reps[b, g]; the partial block (when V mod block != 0) is always kept;
+ *    the best full blocks fill the remaining top_m slots; then the k best of
+ *    the visible entries of the kept blocks are selected.
+ * Ties go to the lower index (entries and blocks).  The idx row holds the
+ * selected entries in ascending order followed by -1 when fewer than k exist.
+ *   qi [batch, T, dI]   q_pos [batch, T] int32   ic [batch, nc_cap, dI]
+ *   reps [batch, nb_cap, dI] with nb_cap >= floor(nc/block) (HISA only)
+ *   idx [batch, T, k] int32
+ * `q_chunk` is the number of queries scored per pass (a scheduling choice;
+ * results do not depend on it; 0 = library default).  Scratch comes from
+ * `ws` (device memory, 256-byte aligned) of at least
+ * hyb_index_topk_workspace_size(...) bytes.
+ */
+size_t hyb_index_topk_workspace_size(int dtype, int batch, int T, int nc, int dI, int k,
+                                     int mode, int block, int top_m, int q_chunk);
+int hyb_index_topk(int dtype, int batch, int T, int dI,
+                   const void* qi, const int* q_pos,
+                   const void* ic, int nc, int nc_cap, int r, int k, int mode,
+                   const void* reps, int nb_cap, int block, int top_m, int q_chunk,
+                   int* idx, void* ws, size_t ws_bytes, hyb_stream_t stream);
+
+/*
+ * S3 + S4 — shared-KV attention with a sliding window (HCA article, section
+ * "怎么压": MQA over all compressed entries (HCA) plus a 128-token window branch,
+ * as in CSA; trdm.cn 2.1: CSA attends the indexer's top-k plus the window).
+ * For query (b, i) at t = q_pos[b, i] and every head h, the key set is
+ *   { compressed entries idx[b, i, :] >= 0 }          (idx != NULL, CSA)
+ *   { compressed entries j < min(floor((t+1)/r), nc) } (idx == NULL, HCA)
+ *  union { raw positions s, max(0, t-W+1) <= s <= t } read from slot s mod ring
+ * of kw / vw, under ONE softmax of scale * q . key:
+ *   o[b, i, h] = sum p v,  lse[b, i, h] = natural log of the softmax denominator.
+ *   q [batch, T, H, D]   kc, vc [batch, nc_cap, D]   idx [batch, T, k] or NULL
+ *   kw, vw [batch, ring, D] (prefill: the raw K/V with ring = L; decode: a
+ *   ring of at least W slots)   o [batch, T, H, D]   lse [batch, T, H] fp32 or NULL
+ * `mode` picks the schedule (HYB_ATTN_DECODE splits each query's keys over
+ * several CTAs and merges the partial softmaxes); both compute the same
+ * function.  Entries of idx outside [0, V) other than -1 are skipped and
+ * reported as HYB_ERR_DEVICE_CHECK.  Scratch: `ws` of at least
+ * hyb_attn_fwd_workspace_size(...) bytes (may be 0 for PREFILL).
+ */
+size_t hyb_attn_fwd_workspace_size(int dtype, int batch, int T, int H, int D, int k,
+                                   int nc, int W, int mode);
+int hyb_attn_fwd(int dtype, int batch, int T, int H, int D,
+                 const void* q, const int* q_pos,
+                 const void* kc, const void* vc, int nc, int nc_cap, int r,
+                 const int* idx, int k,
+                 const void* kw, const void* vw, int ring, int W, float scale,
+                 void* o, float* lse, int mode,
+                 void* ws, size_t ws_bytes, hyb_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYB_H_ */

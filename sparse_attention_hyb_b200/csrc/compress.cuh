@@ -1,0 +1,128 @@
+// S1 — sequence-axis compression (HCA article, section "怎么压"): every entry is
+// a softmax-weighted sum of the raw rows of its window, the weight of a token
+// being softmax over the window of (its compression logit + the learnable bias
+// of its position in the window).  CSA windows are 2r long at stride r, HCA
+// windows r long without overlap.
+//
+// HBM-bound streaming pass.  One warp owns one entry: it computes the window's
+// weights once (lanes over window positions) and then pools K, V and the
+// indexer keys with them (lanes over channels, 4 channels per lane, so a warp
+// reads a whole 256-byte bf16 row per load).  Consecutive warps own
+// consecutive entries, so the raw rows shared by two overlapping CSA windows
+// are read twice within a few hundred nanoseconds and the second read hits L2.
+#pragma once
+#include "common.cuh"
+
+namespace hyb {
+
+constexpr int kCompressWarps = 4;
+constexpr int kMaxSpan = 256;
+
+template <typename T>
+__device__ __forceinline__ void pool_rows(const T* __restrict__ x, T* __restrict__ out, int C,
+                                          int start, int span, const float* w, int lane) {
+  for (int c = lane * 4; c < C; c += 128) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int p = 0; p < span; ++p) {
+      const float wp = w[p];
+      if (wp == 0.f) continue;  // token before the start of the sequence
+      const float4 v = load4(x + (size_t)(start + p) * C + c);
+      acc.x = fmaf(wp, v.x, acc.x);
+      acc.y = fmaf(wp, v.y, acc.y);
+      acc.z = fmaf(wp, v.z, acc.z);
+      acc.w = fmaf(wp, v.w, acc.w);
+    }
+    store4(out + c, acc);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kCompressWarps * 32)
+compress_kernel(const T* __restrict__ xk, const T* __restrict__ xv, const T* __restrict__ xi,
+                const float* __restrict__ logits, const float* __restrict__ bias,
+                T* __restrict__ kc, T* __restrict__ vc, T* __restrict__ ic,
+                int L, int D, int dI, int r, int overlap, int j_begin, int j_end, int nc_cap) {
+  __shared__ float wts[kCompressWarps][kMaxSpan];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int j = j_begin + blockIdx.x * kCompressWarps + warp;
+  if (j >= j_end) return;
+  const int span = overlap ? 2 * r : r;
+  const int start = overlap ? (j - 1) * r : j * r;
+  const float* zb = logits + (size_t)b * L;
+  float* w = wts[warp];
+
+  // Weights: softmax over the in-range tokens of the window.
+  float mx = -INFINITY;
+  for (int p = lane; p < span; p += 32) {
+    const int s = start + p;
+    const float a = s >= 0 ? zb[s] + bias[p] : -INFINITY;
+    w[p] = a;
+    mx = fmaxf(mx, a);
+  }
+  mx = warp_max(mx);
+  float sum = 0.f;
+  for (int p = lane; p < span; p += 32) {
+    const float e = w[p] == -INFINITY ? 0.f : __expf(w[p] - mx);
+    w[p] = e;
+    sum += e;
+  }
+  sum = warp_sum(sum);
+  const float inv = 1.f / sum;
+  for (int p = lane; p < span; p += 32) w[p] *= inv;
+  __syncwarp();
+
+  const size_t row0 = (size_t)b * L;
+  const size_t out0 = (size_t)b * nc_cap + j;
+  pool_rows(xk + row0 * D, kc + out0 * D, D, start, span, w, lane);
+  pool_rows(xv + row0 * D, vc + out0 * D, D, start, span, w, lane);
+  if (xi != nullptr) pool_rows(xi + row0 * dI, ic + out0 * dI, dI, start, span, w, lane);
+}
+
+template <typename T>
+cudaError_t launch_compress(int batch, int L, int D, int dI, const void* xk, const void* xv,
+                            const void* xi, const float* logits, const float* bias, int r,
+                            int overlap, int j_begin, int j_end, void* kc, void* vc, void* ic,
+                            int nc_cap, cudaStream_t stream) {
+  const int n = j_end - j_begin;
+  if (n <= 0 || batch <= 0) return cudaSuccess;
+  dim3 grid((n + kCompressWarps - 1) / kCompressWarps, batch);
+  compress_kernel<T><<<grid, kCompressWarps * 32, 0, stream>>>(
+      (const T*)xk, (const T*)xv, (const T*)xi, logits, bias, (T*)kc, (T*)vc, (T*)ic, L, D, dI, r,
+      overlap, j_begin, j_end, nc_cap);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// HISA block representatives: the mean of the indexer keys of a full block.
+template <typename T>
+__global__ void block_reps_kernel(const T* __restrict__ ic, T* __restrict__ reps, int dI,
+                                  int nc_cap, int block, int g_begin, int nb_cap) {
+  const int g = g_begin + blockIdx.x, b = blockIdx.y;
+  const T* src = ic + ((size_t)b * nc_cap + (size_t)g * block) * dI;
+  const float inv = 1.f / (float)block;
+  for (int c = threadIdx.x * 4; c < dI; c += blockDim.x * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = 0; e < block; ++e) {
+      const float4 v = load4(src + (size_t)e * dI + c);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+    store4(reps + ((size_t)b * nb_cap + g) * dI + c, acc);
+  }
+}
+
+template <typename T>
+cudaError_t launch_block_reps(int batch, int dI, const void* ic, int nc_cap, int block, int g_begin,
+                              int g_end, void* reps, int nb_cap, cudaStream_t stream) {
+  const int n = g_end - g_begin;
+  if (n <= 0 || batch <= 0) return cudaSuccess;
+  const int threads = dI / 4 < 32 ? 32 : (dI / 4 > 256 ? 256 : dI / 4);
+  block_reps_kernel<T><<<dim3(n, batch), threads, 0, stream>>>((const T*)ic, (T*)reps, dI, nc_cap,
+                                                               block, g_begin, nb_cap);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace hyb

@@ -1,0 +1,294 @@
+// libhyb — C ABI entry points (declared and documented in include/hyb.h).
+// Host side: argument checks, workspace carving, launch configuration.  The
+// kernels live in the *.cuh files of this directory; this is the only
+// translation unit, so the per-device status word has a single definition.
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "compress.cuh"
+#include "topk.cuh"
+#include "index.cuh"
+#include "attn.cuh"
+
+using namespace hyb;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+inline bool dtype_ok(int dtype) { return dtype == HYB_DTYPE_F32 || dtype == HYB_DTYPE_BF16; }
+inline size_t dtype_size(int dtype) { return dtype == HYB_DTYPE_F32 ? 4 : 2; }
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA; }
+
+constexpr size_t kSmemTopkMax = 200 * 1024;  // keys staged in shared memory per row
+constexpr size_t kScoreBudget = 64ull << 20; // target bytes of one chunk of scores
+
+// Queries scored per pass so that one chunk of scores stays near kScoreBudget.
+int default_chunk(int batch, int T, size_t row_bytes) {
+  size_t rows = kScoreBudget / (row_bytes * (size_t)batch);
+  if (rows < 64) rows = 64;
+  rows = rows / 64 * 64;
+  return (int)(rows < (size_t)T ? rows : (size_t)T);
+}
+
+struct IndexPlan {
+  int nq;        // queries per chunk (per batch)
+  int ldS;       // flat: score row stride; HISA: block-score row stride
+  int nb;        // HISA: blocks with a representative
+  size_t off_scores, off_blk, off_ncand, off_cand, off_keys, total;
+  bool global_keys;
+};
+
+IndexPlan plan_index(int dtype, int batch, int T, int nc, int k, int mode, int block, int top_m,
+                     int q_chunk) {
+  (void)dtype;
+  IndexPlan p{};
+  if (mode == HYB_INDEX_FLAT) {
+    p.ldS = round_up(nc > 0 ? nc : 1, 4);
+    p.nq = q_chunk > 0 ? (q_chunk < T ? q_chunk : T) : default_chunk(batch, T, (size_t)p.ldS * 4);
+    p.global_keys = (size_t)nc * 4 > kSmemTopkMax;
+    size_t off = 0;
+    p.off_scores = off; off += align_up((size_t)batch * p.nq * p.ldS * 4);
+    p.off_keys = off;   off += p.global_keys ? align_up((size_t)batch * p.nq * p.ldS * 4) : 0;
+    p.total = off;
+  } else {
+    p.nb = nc / block;
+    p.ldS = round_up(p.nb > 0 ? p.nb : 1, 4);
+    const size_t cand = (size_t)top_m * block;
+    p.nq = q_chunk > 0 ? (q_chunk < T ? q_chunk : T) : default_chunk(batch, T, cand * 4 + (size_t)p.ldS * 4);
+    size_t off = 0;
+    p.off_scores = off; off += align_up((size_t)batch * p.nq * p.ldS * 4);
+    p.off_blk = off;    off += align_up((size_t)batch * p.nq * top_m * 4);
+    p.off_ncand = off;  off += align_up((size_t)batch * p.nq * 4);
+    p.off_cand = off;   off += align_up((size_t)batch * p.nq * cand * 4);
+    p.total = off;
+  }
+  return p;
+}
+
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <typename T>
+int index_topk_impl(int batch, int T_, int dI, const void* qi, const int* q_pos, const void* ic,
+                    int nc, int nc_cap, int r, int k, int mode, const void* reps, int nb_cap,
+                    int block, int top_m, const IndexPlan& p, int* idx, char* ws,
+                    cudaStream_t stream) {
+  cudaError_t e = cudaSuccess;
+  float* S = reinterpret_cast<float*>(ws + p.off_scores);
+  for (int i0 = 0; i0 < T_; i0 += p.nq) {
+    const int nq = T_ - i0 < p.nq ? T_ - i0 : p.nq;
+    if (mode == HYB_INDEX_FLAT) {
+      dim3 g((nc + kSB_N - 1) / kSB_N, (nq + kSB_M - 1) / kSB_M, batch);
+      if (nc > 0) {
+        scores_ffma_kernel<T><<<g, 256, 0, stream>>>((const T*)qi, q_pos, (const T*)ic, S, T_, i0, nq,
+                                                     dI, nc_cap, r, nc, 1, p.ldS);
+        count_launch();
+      }
+      const size_t smem = p.global_keys ? 0 : (size_t)nc * 4;
+      if ((e = allow_smem(select_flat_kernel, smem)) != cudaSuccess) return HYB_ERR_CUDA;
+      uint32_t* gkeys = p.global_keys ? reinterpret_cast<uint32_t*>(ws + p.off_keys) : nullptr;
+      select_flat_kernel<<<dim3(nq, batch), kTopkThreads, smem, stream>>>(S, q_pos, idx, T_, i0, nq, r,
+                                                                          nc, k, p.ldS, gkeys);
+      count_launch();
+    } else {
+      int* blk = reinterpret_cast<int*>(ws + p.off_blk);
+      int* ncand = reinterpret_cast<int*>(ws + p.off_ncand);
+      float* SC = reinterpret_cast<float*>(ws + p.off_cand);
+      if (p.nb > 0) {
+        dim3 g((p.nb + kSB_N - 1) / kSB_N, (nq + kSB_M - 1) / kSB_M, batch);
+        scores_ffma_kernel<T><<<g, 256, 0, stream>>>((const T*)qi, q_pos, (const T*)reps, S, T_, i0, nq,
+                                                     dI, nb_cap, r, nc, block, p.ldS);
+      count_launch();
+      }
+      const size_t smem1 = (size_t)(p.nb > 0 ? p.nb : 1) * 4;
+      if ((e = allow_smem(select_blocks_kernel, smem1)) != cudaSuccess) return HYB_ERR_CUDA;
+      select_blocks_kernel<<<dim3(nq, batch), kTopkThreads, smem1, stream>>>(S, q_pos, blk, T_, i0, nq, r,
+                                                                             nc, block, top_m, p.ldS);
+      count_launch();
+      hisa_cand_scores_kernel<T><<<dim3(nq, batch), 256, dI * 4, stream>>>(
+          (const T*)qi, q_pos, (const T*)ic, blk, SC, ncand, T_, i0, nq, dI, nc_cap, r, nc, block, top_m);
+      count_launch();
+      const size_t smem2 = (size_t)top_m * block * 4;
+      if ((e = allow_smem(select_cand_kernel, smem2)) != cudaSuccess) return HYB_ERR_CUDA;
+      select_cand_kernel<<<dim3(nq, batch), kTopkThreads, smem2, stream>>>(SC, ncand, blk, idx, T_, i0, nq,
+                                                                           block, top_m, k);
+      count_launch();
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return HYB_ERR_CUDA;
+  }
+  return HYB_OK;
+}
+
+int attn_splits(int mode, int batch, int T, int n_keys_max) {
+  if (mode != HYB_ATTN_DECODE) return 1;
+  // enough CTAs to cover the SMs a few times, at least 64 keys per split
+  const int ctas = batch * T;
+  int ns = (4 * 148 + ctas - 1) / ctas;
+  const int cap = (n_keys_max + 63) / 64;
+  if (ns > cap) ns = cap;
+  if (ns < 1) ns = 1;
+  if (ns > 64) ns = 64;
+  return ns;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* hyb_status_string(int status) {
+  switch (status) {
+    case HYB_OK: return "HYB_OK";
+    case HYB_ERR_INVALID_ARG: return "HYB_ERR_INVALID_ARG: invalid argument";
+    case HYB_ERR_UNSUPPORTED: return "HYB_ERR_UNSUPPORTED: dtype, size or alignment not supported";
+    case HYB_ERR_WORKSPACE: return "HYB_ERR_WORKSPACE: workspace missing or too small";
+    case HYB_ERR_CUDA: return "HYB_ERR_CUDA: CUDA launch or runtime call failed";
+    case HYB_ERR_TIMEOUT: return "HYB_ERR_TIMEOUT: a bounded device wait gave up";
+    case HYB_ERR_DEVICE_CHECK: return "HYB_ERR_DEVICE_CHECK: a device-side index or size check failed";
+    default: return "HYB_ERR_UNKNOWN";
+  }
+}
+
+int hyb_abi_version(void) { return 100; }
+
+unsigned long long hyb_kernel_launches(void) { return launch_counter().load(); }
+
+int hyb_get_device_status(hyb_stream_t stream, int* status) {
+  if (!status) return HYB_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int host = 0;
+  const int zero = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HYB_ERR_CUDA;
+  if (cudaMemcpyFromSymbolAsync(&host, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return HYB_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return HYB_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HYB_ERR_CUDA;
+  *status = host;
+  return HYB_OK;
+}
+
+int hyb_compress(int dtype, int batch, int L, int D, int dI, const void* xk, const void* xv,
+                 const void* xi, const float* logits, const float* bias, int r, int overlap,
+                 int j_begin, int j_end, void* kc, void* vc, void* ic, int nc_cap,
+                 hyb_stream_t stream) {
+  if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
+  if (batch < 0 || L < 0 || D <= 0 || r < 1 || j_begin < 0 || j_end < j_begin || nc_cap < j_end)
+    return HYB_ERR_INVALID_ARG;
+  if ((long long)j_end * r > L) return HYB_ERR_INVALID_ARG;
+  if (!xk || !xv || !logits || !bias || !kc || !vc) return HYB_ERR_INVALID_ARG;
+  if (xi && (!ic || dI <= 0)) return HYB_ERR_INVALID_ARG;
+  const int span = overlap ? 2 * r : r;
+  if (span > kMaxSpan || D % 4 != 0 || (xi && dI % 4 != 0)) return HYB_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = dtype == HYB_DTYPE_F32
+      ? launch_compress<float>(batch, L, D, dI, xk, xv, xi, logits, bias, r, overlap ? 1 : 0, j_begin,
+                               j_end, kc, vc, ic, nc_cap, s)
+      : launch_compress<bf16>(batch, L, D, dI, xk, xv, xi, logits, bias, r, overlap ? 1 : 0, j_begin,
+                              j_end, kc, vc, ic, nc_cap, s);
+  return cuda_status(e);
+}
+
+int hyb_block_reps(int dtype, int batch, int dI, const void* ic, int nc_cap, int block, int g_begin,
+                   int g_end, void* reps, int nb_cap, hyb_stream_t stream) {
+  if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
+  if (batch < 0 || dI <= 0 || block < 1 || g_begin < 0 || g_end < g_begin || g_end > nb_cap ||
+      (long long)g_end * block > nc_cap)
+    return HYB_ERR_INVALID_ARG;
+  if (!ic || !reps) return HYB_ERR_INVALID_ARG;
+  if (dI % 4 != 0) return HYB_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = dtype == HYB_DTYPE_F32
+      ? launch_block_reps<float>(batch, dI, ic, nc_cap, block, g_begin, g_end, reps, nb_cap, s)
+      : launch_block_reps<bf16>(batch, dI, ic, nc_cap, block, g_begin, g_end, reps, nb_cap, s);
+  return cuda_status(e);
+}
+
+size_t hyb_index_topk_workspace_size(int dtype, int batch, int T, int nc, int dI, int k, int mode,
+                                     int block, int top_m, int q_chunk) {
+  (void)dI;
+  if (batch <= 0 || T <= 0 || nc < 0 || k < 1) return 0;
+  if (mode == HYB_INDEX_HISA && (block < 1 || top_m < 1)) return 0;
+  return plan_index(dtype, batch, T, nc, k, mode, block, top_m, q_chunk).total;
+}
+
+int hyb_index_topk(int dtype, int batch, int T, int dI, const void* qi, const int* q_pos,
+                   const void* ic, int nc, int nc_cap, int r, int k, int mode, const void* reps,
+                   int nb_cap, int block, int top_m, int q_chunk, int* idx, void* ws,
+                   size_t ws_bytes, hyb_stream_t stream) {
+  if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
+  if (mode != HYB_INDEX_FLAT && mode != HYB_INDEX_HISA) return HYB_ERR_INVALID_ARG;
+  if (batch < 0 || T < 0 || dI <= 0 || nc < 0 || nc_cap < nc || r < 1 || k < 1 || q_chunk < 0)
+    return HYB_ERR_INVALID_ARG;
+  if (batch == 0 || T == 0) return HYB_OK;
+  if (!qi || !q_pos || !ic || !idx) return HYB_ERR_INVALID_ARG;
+  if (dI % 4 != 0) return HYB_ERR_UNSUPPORTED;
+  if (mode == HYB_INDEX_HISA) {
+    if (block < 1 || top_m < 1 || !reps || nb_cap < nc / block) return HYB_ERR_INVALID_ARG;
+    if ((size_t)top_m * block * 4 > kSmemTopkMax || (size_t)(nc / block) * 4 > kSmemTopkMax)
+      return HYB_ERR_UNSUPPORTED;
+  }
+  const IndexPlan p = plan_index(dtype, batch, T, nc, k, mode, block, top_m, q_chunk);
+  if (!ws || ws_bytes < p.total || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return HYB_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  return dtype == HYB_DTYPE_F32
+      ? index_topk_impl<float>(batch, T, dI, qi, q_pos, ic, nc, nc_cap, r, k, mode, reps, nb_cap, block,
+                               top_m, p, idx, w, s)
+      : index_topk_impl<bf16>(batch, T, dI, qi, q_pos, ic, nc, nc_cap, r, k, mode, reps, nb_cap, block,
+                              top_m, p, idx, w, s);
+}
+
+size_t hyb_attn_fwd_workspace_size(int dtype, int batch, int T, int H, int D, int k, int nc, int W,
+                                   int mode) {
+  (void)dtype;
+  if (batch <= 0 || T <= 0 || H <= 0 || D <= 0) return 0;
+  const int n_keys = (k > 0 ? k : nc) + W;
+  const int ns = attn_splits(mode, batch, T, n_keys);
+  if (ns <= 1) return 0;
+  const size_t rows = (size_t)batch * T * ns * H;
+  return align_up(rows * D * 4) + align_up(rows * 4);
+}
+
+int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const int* q_pos,
+                 const void* kc, const void* vc, int nc, int nc_cap, int r, const int* idx, int k,
+                 const void* kw, const void* vw, int ring, int W, float scale, void* o, float* lse,
+                 int mode, void* ws, size_t ws_bytes, hyb_stream_t stream) {
+  if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
+  if (mode != HYB_ATTN_PREFILL && mode != HYB_ATTN_DECODE) return HYB_ERR_INVALID_ARG;
+  if (batch < 0 || T < 0 || H <= 0 || D <= 0 || nc < 0 || nc_cap < nc || r < 1 || W < 0 ||
+      (idx && k < 1) || ring < 1 || ring < W)
+    return HYB_ERR_INVALID_ARG;
+  if (batch == 0 || T == 0) return HYB_OK;
+  if (!q || !q_pos || !kw || !vw || !o || ((nc > 0) && (!kc || !vc))) return HYB_ERR_INVALID_ARG;
+  if (!attn_ffma_supported(H, D)) return HYB_ERR_UNSUPPORTED;
+  const int n_keys = (idx ? k : nc) + W;
+  const int ns = attn_splits(mode, batch, T, n_keys);
+  AttnArgs a{q, q_pos, kc, vc, nc, nc_cap, r, idx, k, kw, vw, ring, W, scale, o, lse,
+             nullptr, nullptr, T, H, D, ns};
+  if (ns > 1) {
+    const size_t rows = (size_t)batch * T * ns * H;
+    const size_t need = align_up(rows * D * 4) + align_up(rows * 4);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return HYB_ERR_WORKSPACE;
+    a.part_o = static_cast<float*>(ws);
+    a.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + align_up(rows * D * 4));
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dtype == HYB_DTYPE_F32) {
+    if ((e = launch_attn_ffma<float>(a, batch, s)) != cudaSuccess) return HYB_ERR_CUDA;
+    if (ns > 1) { attn_merge_kernel<float><<<dim3(batch * T, H), 128, 0, s>>>(a); count_launch(); }
+  } else {
+    if ((e = launch_attn_ffma<bf16>(a, batch, s)) != cudaSuccess) return HYB_ERR_CUDA;
+    if (ns > 1) { attn_merge_kernel<bf16><<<dim3(batch * T, H), 128, 0, s>>>(a); count_launch(); }
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

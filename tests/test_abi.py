@@ -1,0 +1,76 @@
+"""The C ABI without a GPU: libhyb.so loads, exports every entry point that
+include/hyb.h declares, and rejects bad arguments on the host before any
+launch (these paths touch no CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def A():
+    from sparse_attention_hyb_b200 import abi, build
+    build.build()
+    abi.lib()
+    return abi
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "hyb.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hyb_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(A):
+    names = _declared()
+    assert len(names) >= 9
+    lib = ctypes.CDLL(A.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in A.SIGNATURES, f"binding lacks {n}"
+
+
+def test_status_strings_and_version(A):
+    assert A.hyb_abi_version() == 100
+    for code in range(7):
+        assert A.status_string(code).startswith("HYB_")
+    assert A.status_string(99) == "HYB_ERR_UNKNOWN"
+
+
+def test_host_argument_checks(A):
+    L = A.lib()
+    # unsupported dtype, null pointers, inconsistent ranges: rejected before any launch
+    assert L.hyb_compress(7, 1, 8, 4, 4, 1, 1, None, 1, 1, 4, 1, 0, 1, 1, 1, None, 2, None) == A.HYB_ERR_UNSUPPORTED
+    assert L.hyb_compress(1, 1, 8, 4, 4, None, 1, None, 1, 1, 4, 1, 0, 1, 1, 1, None, 2, None) == A.HYB_ERR_INVALID_ARG
+    assert L.hyb_compress(1, 1, 8, 4, 4, 1, 1, None, 1, 1, 4, 1, 0, 3, 1, 1, None, 3, None) == A.HYB_ERR_INVALID_ARG
+    assert L.hyb_compress(1, 1, 1024, 4, 4, 1, 1, None, 1, 1, 200, 1, 0, 1, 1, 1, None, 1, None) == A.HYB_ERR_UNSUPPORTED
+    assert L.hyb_compress(1, 1, 8, 6, 4, 1, 1, None, 1, 1, 4, 1, 0, 1, 1, 1, None, 2, None) == A.HYB_ERR_UNSUPPORTED
+    assert L.hyb_block_reps(1, 1, 128, 1, 100, 128, 0, 1, 1, 1, None) == A.HYB_ERR_INVALID_ARG
+    # index: bad mode, missing workspace, HISA without representatives
+    args = [1, 1, 16, 128, 1, 1, 1, 64, 64, 4, 8]
+    assert L.hyb_index_topk(*args, 5, None, 0, 0, 0, 0, 1, None, 0, None) == A.HYB_ERR_INVALID_ARG
+    assert L.hyb_index_topk(*args, 0, None, 0, 0, 0, 0, 1, None, 0, None) == A.HYB_ERR_WORKSPACE
+    assert L.hyb_index_topk(*args, 1, None, 0, 16, 4, 0, 1, 256, 1 << 20, None) == A.HYB_ERR_INVALID_ARG
+    assert L.hyb_index_topk(*args, 0, None, 0, 0, 0, 0, 1, 256 + 8, 1 << 30, None) == A.HYB_ERR_WORKSPACE
+    # attention: ring smaller than the window, unsupported head geometry, missing workspace
+    a = [1, 1, 4, 64, 128, 1, 1, 1, 1, 10, 10, 4, None, 0, 1, 1]
+    assert L.hyb_attn_fwd(*a, 64, 128, ctypes.c_float(0.1), 1, None, 0, None, 0, None) == A.HYB_ERR_INVALID_ARG
+    b = [1, 1, 4, 48, 128, 1, 1, 1, 1, 10, 10, 4, None, 0, 1, 1]
+    assert L.hyb_attn_fwd(*b, 128, 128, ctypes.c_float(0.1), 1, None, 0, None, 0, None) == A.HYB_ERR_UNSUPPORTED
+    assert L.hyb_attn_fwd(*a, 128, 128, ctypes.c_float(0.1), 1, None, 1, None, 0, None) == A.HYB_ERR_WORKSPACE
+    # empty problems are fine and launch nothing
+    assert L.hyb_attn_fwd(1, 0, 4, 64, 128, None, None, None, None, 0, 0, 4, None, 0, None, None, 128, 128,
+                          ctypes.c_float(0.1), None, None, 0, None, 0, None) == A.HYB_OK
+
+
+def test_workspace_sizes(A):
+    f = A.hyb_index_topk_workspace_size
+    flat = f(1, 1, 32768, 8192, 128, 512, A.HYB_INDEX_FLAT)
+    assert flat >= 64 * 8192 * 4 and flat % 256 == 0
+    hisa = f(1, 1, 131072, 32768, 128, 2048, A.HYB_INDEX_HISA, 128, 64, 1024)
+    assert hisa >= 1024 * 64 * 128 * 4
+    assert A.hyb_attn_fwd_workspace_size(1, 1, 32768, 64, 128, 512, 8192, 128, A.HYB_ATTN_PREFILL) == 0
+    assert A.hyb_attn_fwd_workspace_size(1, 64, 1, 64, 128, 512, 32768, 128, A.HYB_ATTN_DECODE) > 0

@@ -1,0 +1,243 @@
+"""GPU parity of the whole layer on the five workloads, against the fp64 oracle.
+
+The GPU runs every query of a workload in the same launch configuration as
+the benchmark; the oracle recomputes a seeded sample of rows (always the first
+and last rows, rows next to compression and block boundaries, and queries that
+carry a planted key) from the same generated inputs, including its own S1 pass
+over the raw sequence.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from workloads import configs as C
+from workloads import make
+
+from parity import (BF16_REL_L2, IOU_MIN, check_close, sample_rows, to64, topk_row_check)
+
+pytestmark = pytest.mark.gpu
+dev = "cuda"
+
+
+@pytest.fixture(scope="module")
+def S():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import sparse_attention_hyb_b200 as S
+    S.abi.lib()
+    return S
+
+
+@pytest.fixture(autouse=True)
+def _status_clean(S):
+    S.abi.hyb_get_device_status()
+    yield
+    assert S.abi.hyb_get_device_status() == 0
+
+
+def _params(w, ly):
+    return O.LayerParams(ly.kind, ly.r, ly.overlap, w.W, 1.0 / math.sqrt(w.D), w.dtype, k=ly.k,
+                         index_mode=ly.index_mode, block=ly.block, top_m=ly.top_m)
+
+
+def _gpu_layer(S, w, ly, raw_d, qs_d, bias_d, n_c, ring_k, ring_v, mode, rows=None):
+    """S1 (whole prefix) + S2 + S3 on the device; returns dict of device tensors."""
+    xi = raw_d.get("xi") if ly.kind == "csa" else None
+    kc, vc, ic = S.layer.compress(raw_d["xk"], raw_d["xv"], xi, raw_d["z"], bias_d, ly.r, ly.overlap, n_c)
+    q, qi, q_pos = qs_d["q"], qs_d["qi"], qs_d["q_pos"]
+    if rows is not None:
+        q, qi, q_pos = q[:, rows].contiguous(), qi[:, rows].contiguous(), q_pos[:, rows].contiguous()
+    out = {"kc": kc, "vc": vc, "ic": ic, "idx": None, "reps": None, "qi": qi, "q_pos": q_pos}
+    if ly.kind == "csa":
+        if ly.index_mode == "hisa":
+            out["reps"] = S.layer.block_reps(ic, n_c, ly.block)
+            out["idx"] = S.layer.index_topk(qi, q_pos, ic, n_c, ly.r, ly.k, S.HYB_INDEX_HISA, out["reps"],
+                                            ly.block, ly.top_m, ly.q_chunk)
+        else:
+            out["idx"] = S.layer.index_topk(qi, q_pos, ic, n_c, ly.r, ly.k)
+    md = S.HYB_ATTN_DECODE if mode == "decode" else S.HYB_ATTN_PREFILL
+    out["o"], out["lse"] = S.layer.attention(q, q_pos, kc, vc, n_c, ly.r, out["idx"], ring_k, ring_v, w.W,
+                                             1.0 / math.sqrt(w.D), md)
+    torch.cuda.synchronize()
+    return out
+
+
+def _compare_rows(w, ly, p, gpu, b, rows, q, qi, q_pos, caches, ring_k, ring_v, ring, gpu_rows=None,
+                  planted=()):
+    """Oracle rows vs GPU rows.  Returns (iou list, matched-row o pairs, all-row o pairs)."""
+    kc, vc, ic, reps = caches
+    gidx = gpu["idx"][b].cpu().numpy() if gpu["idx"] is not None else None
+    go = to64(gpu["o"][b])
+    gl = to64(gpu["lse"][b])
+    ious, matched, allp = [], [], []
+    for n, i in enumerate(rows):
+        gi = n if gpu_rows is not None else i
+        t = int(q_pos[i])
+        idx, o, l = O.layer_row(p, q[i], qi[i] if qi is not None else None, t, kc, vc, ic, reps, ring_k,
+                                ring_v, ring)
+        same = True
+        if idx is not None:
+            n_vis = O.visible_entries(t, ly.r, kc.shape[0])
+            if ly.index_mode == "flat":
+                ids = np.arange(n_vis)
+            else:
+                blocks = O.hisa_blocks(qi[i], reps, n_vis, ly.block, ly.top_m)
+                ids = np.concatenate([np.arange(g * ly.block, min((g + 1) * ly.block, n_vis)) for g in blocks]) \
+                    if len(blocks) else np.empty(0, dtype=np.int64)
+            s = O.index_scores(qi[i], ic, ids)
+            eps = 2 * qi.shape[1] * 2.0 ** -24 * (np.abs(ic[ids]) @ np.abs(qi[i])) + \
+                (np.abs(qi[i]) @ (2.0 ** -7 * np.abs(ic[ids]).T) if w.dtype == "bf16" else 0.0)
+            iou, _ = topk_row_check(gidx[gi], s, ids, ly.k, eps, f"{w.name} row {i}")
+            ious.append(iou)
+            same = set(gidx[gi][gidx[gi] >= 0].tolist()) == set(idx[idx >= 0].tolist())
+            for j in planted:
+                if j < n_vis and np.dot(qi[i], ic[j]) > 0.4 * np.linalg.norm(qi[i]) * np.linalg.norm(ic[j]):
+                    assert j in set(gidx[gi].tolist()), f"planted entry {j} missed by row {i}"
+        allp.append((go[gi], o))
+        if same:
+            matched.append((go[gi], o))
+            np.testing.assert_allclose(gl[gi], l, atol=1e-3 if w.dtype == "bf16" else 1e-4, rtol=0)
+    return ious, matched, allp
+
+
+def _assert_outputs(w, matched, allp, min_matched=0.9):
+    assert len(matched) >= min_matched * len(allp), f"only {len(matched)}/{len(allp)} rows with identical idx"
+    check_close(np.stack([g for g, _ in matched]), np.stack([o for _, o in matched]), w.dtype, f"{w.name} o")
+    if w.dtype == "bf16":
+        g, o = np.stack([g for g, _ in allp]), np.stack([o for _, o in allp])
+        assert np.linalg.norm(g - o) / np.linalg.norm(o) <= BF16_REL_L2
+
+
+def _prefill_case(S, w, ly, n_rows, seed, gpu_rows=None):
+    raw, qs = make.make_raw(w), make.make_queries(w)
+    planted = make.plant_prefill(w, ly, raw, qs).tolist()
+    bias = make.make_bias(w, ly)
+    raw_d = {k: v.to(dev) for k, v in raw.items()}
+    qs_d = {k: v.to(dev) for k, v in qs.items()}
+    L = raw["xk"].shape[1]
+    n_c = L // ly.r
+    gpu = _gpu_layer(S, w, ly, raw_d, qs_d, bias.to(dev), n_c, raw_d["xk"], raw_d["xv"], "prefill", gpu_rows)
+    p = _params(w, ly)
+    xi64 = to64(raw["xi"][0]) if ly.kind == "csa" else None
+    kc, vc, ic = O.build_caches(p, to64(raw["xk"][0]), to64(raw["xv"][0]), xi64, to64(raw["z"][0]),
+                                to64(bias), n_c)
+    reps = O.block_reps(ic, ly.block, w.dtype) if ly.index_mode == "hisa" and ly.kind == "csa" else None
+    extra = [4 * j + 3 for j in planted[:8]] + [ly.r * 64 - 1, ly.r * 64, 127, 128, 129]
+    extra = [x - w.q_pos0 for x in extra]
+    if gpu_rows is None:
+        rows = sample_rows(w.T, n_rows, seed, extra)
+    else:
+        rows = np.asarray(gpu_rows)
+    q64 = {int(i): to64(qs["q"][0, i]) for i in rows}
+    qi64 = to64(qs["qi"][0]) if ly.kind == "csa" else None
+    class Q:  # lazy row access without converting the whole q tensor
+        def __getitem__(self, i):
+            return q64[int(i)]
+    res = _compare_rows(w, ly, p, gpu, 0, rows, Q(), qi64, qs["q_pos"][0].numpy(), (kc, vc, ic, reps),
+                        to64(raw["xk"][0]), to64(raw["xv"][0]), L, gpu_rows, planted)
+    return gpu, res
+
+
+def test_tiny_f32_both_layers(S):
+    w = C.TINY
+    for ly in w.layers:
+        gpu, (ious, matched, allp) = _prefill_case(S, w, ly, w.T, 0)
+        if ly.kind == "csa":
+            assert np.mean(ious) >= IOU_MIN
+        _assert_outputs(w, matched, allp, min_matched=0.99)
+        assert len(allp) == w.T
+
+
+def test_csa_prefill_32k(S):
+    w = C.PREFILL_32K
+    gpu, (ious, matched, allp) = _prefill_case(S, w, w.layer("csa"), 160, 1)
+    assert np.mean(ious) >= IOU_MIN
+    _assert_outputs(w, matched, allp)
+
+
+def test_csa_prefill_128k_hisa_vs_flat(S):
+    w = C.PREFILL_128K
+    ly = w.layer("csa")
+    gpu, (ious, matched, allp) = _prefill_case(S, w, ly, 48, 2)
+    assert np.mean(ious) >= IOU_MIN
+    _assert_outputs(w, matched, allp)
+    # flat selection on the same device caches, for the HISA-vs-flat IoU report
+    flat = S.layer.index_topk(gpu["qi"], gpu["q_pos"], gpu["ic"], gpu["ic"].shape[1], ly.r, ly.k)
+    torch.cuda.synchronize()
+    a, b = gpu["idx"][0].cpu().numpy(), flat[0].cpu().numpy()
+    rows = np.arange(0, w.T, 97)
+    iou = np.mean([len(set(a[i]) & set(b[i]) - {-1}) / max(1, len(set(a[i]) | set(b[i]) - {-1})) for i in rows])
+    print(f"HISA vs flat selection IoU over {len(rows)} rows: {iou:.4f}")
+    assert 0.0 < iou <= 1.0
+
+
+def test_decode_bs64_128k(S):
+    w = C.DECODE_BS64_128K
+    qs = make.make_queries(w)
+    cache = make.make_decode_cache(w)
+    planted = make.plant_decode(w, w.layer("csa"), cache, qs)
+    qs_d = {k: v.to(dev) for k, v in qs.items()}
+    cd = {k: v.to(dev) for k, v in cache.items()}
+    scale = 1.0 / math.sqrt(w.D)
+    for ly in w.layers:
+        n_c = w.L // ly.r
+        kc, vc = cd[f"kc_{ly.kind}"], cd[f"vc_{ly.kind}"]
+        idx = S.layer.index_topk(qs_d["qi"], qs_d["q_pos"], cd["ic"], n_c, ly.r, ly.k) if ly.kind == "csa" else None
+        o, lse = S.layer.attention(qs_d["q"], qs_d["q_pos"], kc, vc, n_c, ly.r, idx, cd["kw"], cd["vw"], w.W,
+                                   scale, S.HYB_ATTN_DECODE)
+        torch.cuda.synchronize()
+        p = _params(w, ly)
+        ious, matched, allp = [], [], []
+        for b in (0, 1, 2, 17, 40, 63):
+            ic64 = to64(cache["ic"][b]) if ly.kind == "csa" else None
+            gpu = {"idx": idx[b:b + 1] if idx is not None else None, "o": o[b:b + 1], "lse": lse[b:b + 1]}
+            res = _compare_rows(w, ly, p, gpu, 0, [0], to64(qs["q"][b]),
+                                to64(qs["qi"][b]) if ly.kind == "csa" else None, qs["q_pos"][b].numpy(),
+                                (to64(cache[f"kc_{ly.kind}"][b]), to64(cache[f"vc_{ly.kind}"][b]), ic64, None),
+                                to64(cache["kw"][b]), to64(cache["vw"][b]), w.W)
+            ious += res[0]
+            matched += res[1]
+            allp += res[2]
+            if ly.kind == "csa":
+                pick = set(idx[b, 0].tolist())
+                assert any(int(j) in pick for j in planted[b].tolist())
+        if ly.kind == "csa":
+            assert np.mean(ious) >= IOU_MIN
+        _assert_outputs(w, matched, allp, min_matched=0.8)
+
+
+def test_ctx_1m_decode(S):
+    w = C.CTX_1M_DECODE
+    raw, qs = make.make_raw(w), make.make_queries(w)
+    planted = make.plant_prefill(w, w.layer("csa"), raw, qs).tolist()
+    raw_d = {k: v.to(dev) for k, v in raw.items()}
+    qs_d = {k: v.to(dev) for k, v in qs.items()}
+    ring = make.ring_from_raw(w, raw)
+    ring_d = {k: v.to(dev) for k, v in ring.items()}
+    for ly in w.layers:
+        bias = make.make_bias(w, ly)
+        n_c = w.L // ly.r
+        gpu = _gpu_layer(S, w, ly, raw_d, qs_d, bias.to(dev), n_c, ring_d["kw"], ring_d["vw"], "decode")
+        p = _params(w, ly)
+        xi64 = to64(raw["xi"][0]) if ly.kind == "csa" else None
+        kc, vc, ic = O.build_caches(p, to64(raw["xk"][0]), to64(raw["xv"][0]), xi64, to64(raw["z"][0]),
+                                    to64(bias), n_c)
+        reps = O.block_reps(ic, ly.block, w.dtype) if ly.kind == "csa" else None
+        ious, matched, allp = _compare_rows(w, ly, p, gpu, 0, [0], to64(qs["q"][0]),
+                                            to64(qs["qi"][0]) if ly.kind == "csa" else None,
+                                            qs["q_pos"][0].numpy(), (kc, vc, ic, reps), to64(ring["kw"][0]),
+                                            to64(ring["vw"][0]), w.W, planted=planted)
+        _assert_outputs(w, matched, allp, min_matched=1.0)
+
+
+def test_ctx_1m_chunk_prefill(S):
+    w = C.CTX_1M_CHUNK
+    for ly in w.layers:
+        rows = None if ly.kind == "csa" else sample_rows(w.T, 200, 3)
+        gpu, (ious, matched, allp) = _prefill_case(S, w, ly, 64, 3, gpu_rows=rows)
+        if ly.kind == "csa":
+            assert np.mean(ious) >= IOU_MIN
+        _assert_outputs(w, matched, allp)

@@ -1,0 +1,242 @@
+"""GPU parity of each libhyb stage against the fp64 oracle on identical seeded
+inputs: several tiles plus ragged tails, both storage types, edge cases
+(nothing visible, fewer candidates than k, partial HISA blocks, split-KV)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from workloads import make, rng
+
+from parity import (acc_bound, check_close, to64, topk_row_check)
+
+pytestmark = pytest.mark.gpu
+
+dev = "cuda"
+
+
+@pytest.fixture(scope="module")
+def S():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import sparse_attention_hyb_b200 as S
+    S.abi.lib()
+    return S
+
+
+@pytest.fixture(autouse=True)
+def _status_clean(S):
+    S.abi.hyb_get_device_status()
+    yield
+    assert S.abi.hyb_get_device_status() == 0
+
+
+def _normal(name, shape, std, dtype, seed=1):
+    return make.normal_tensor(seed, name, shape, std, dtype)
+
+
+def _ulp_bf16(x):
+    a = np.maximum(np.abs(x), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+# --------------------------------------------------------------------------- S1
+
+
+@pytest.mark.parametrize("dtype,B,L,D,dI,r,overlap,j0,j1", [
+    ("f32", 1, 512, 64, 32, 4, True, 0, 128),
+    ("f32", 1, 512, 64, 32, 128, False, 0, 4),
+    ("bf16", 2, 1003, 128, 128, 4, True, 0, 250),
+    ("bf16", 2, 1003, 128, 64, 4, True, 37, 201),
+    ("bf16", 3, 1000, 128, 128, 128, False, 0, 7),
+    ("bf16", 1, 777, 96, 32, 3, True, 0, 259),
+])
+def test_compress(S, dtype, B, L, D, dI, r, overlap, j0, j1):
+    sc = 1.0 if dtype == "f32" else 128 ** -0.5
+    xk, xv = _normal("k", (B, L, D), sc, dtype), _normal("v", (B, L, D), sc, dtype)
+    xi = _normal("i", (B, L, dI), sc, dtype) if overlap else None
+    z = _normal("z", (B, L), 1.0, "f32")
+    bias = _normal("b", (2 * r if overlap else r,), 0.1, "f32")
+    nc = L // r
+    kc = torch.zeros(B, nc, D, dtype=xk.dtype, device=dev)
+    vc, ic = torch.zeros_like(kc), (torch.zeros(B, nc, dI, dtype=xk.dtype, device=dev) if overlap else None)
+    g = lambda t: None if t is None else t.to(dev)
+    S.abi.hyb_compress(g(xk), g(xv), g(xi), g(z), g(bias), r, overlap, j0, j1, kc, vc, ic)
+    torch.cuda.synchronize()
+    for b in range(B):
+        xs = [to64(xk[b]), to64(xv[b])] + ([to64(xi[b])] if overlap else [])
+        want = O.compress(xs, to64(z[b]), to64(bias), r, overlap, j0, j1, dtype)
+        got = [kc[b, j0:j1], vc[b, j0:j1]] + ([ic[b, j0:j1]] if overlap else [])
+        for gt, wt, nm in zip(got, want, "kvi"):
+            g64 = to64(gt)
+            check_close(g64, wt, dtype, f"compress {nm} b={b}")
+            if dtype == "bf16":   # at most one bf16 ulp from the fp64 result rounded once
+                assert np.all(np.abs(g64 - wt) <= _ulp_bf16(wt) * 1.0001), f"{nm}: more than one ulp"
+        assert torch.all(kc[b, :j0] == 0) and torch.all(kc[b, j1:] == 0)   # nothing outside the range
+
+
+def test_block_reps(S):
+    B, nc, dI, blk = 2, 1000, 128, 128
+    ic = _normal("ic", (B, nc, dI), 0.1, "bf16")
+    reps = torch.zeros(B, 8, dI, dtype=torch.bfloat16, device=dev)
+    S.abi.hyb_block_reps(ic.to(dev), blk, 0, nc // blk, reps)
+    torch.cuda.synchronize()
+    for b in range(B):
+        want = O.block_reps(to64(ic[b]), blk, "bf16")
+        got = to64(reps[b, :nc // blk])
+        assert np.all(np.abs(got - want) <= _ulp_bf16(want) * 1.0001)
+    assert torch.all(reps[:, nc // blk:] == 0)
+
+
+# --------------------------------------------------------------------------- S2
+
+
+def _positions(B, T, hi, seed):
+    p = rng.randint_below(seed, "pos", 0, B * T, hi).view(B, T).to(torch.int32)
+    if T >= 8:
+        p[:, :4] = torch.tensor([0, 2, 3, 7], dtype=torch.int32)  # nothing / one entry visible
+        p[:, 4] = hi - 1
+    return p
+
+
+@pytest.mark.parametrize("dtype,B,T,nc,dI,r,k,chunk", [
+    ("f32", 1, 300, 128, 32, 4, 16, 0),
+    ("bf16", 2, 700, 3000, 128, 4, 64, 0),
+    ("bf16", 2, 700, 3000, 128, 4, 64, 128),
+    ("bf16", 64, 1, 8192, 128, 4, 512, 0),
+    ("bf16", 1, 200, 33000, 128, 4, 2048, 0),
+])
+def test_index_flat(S, dtype, B, T, nc, dI, r, k, chunk):
+    sc = 1.0 if dtype == "f32" else dI ** -0.5
+    ic = _normal("ic", (B, nc, dI), sc, dtype)
+    qi = _normal("qi", (B, T, dI), sc, dtype)
+    q_pos = _positions(B, T, r * nc + 40, 5)
+    idx = S.layer.index_topk(qi.to(dev), q_pos.to(dev), ic.to(dev), nc, r, k, q_chunk=chunk)
+    torch.cuda.synchronize()
+    idx = idx.cpu().numpy()
+    ious = []
+    for b in range(B):
+        ic64, qi64 = to64(ic[b]), to64(qi[b])
+        for i in range(T):
+            t = int(q_pos[b, i])
+            n = O.visible_entries(t, r, nc)
+            ids = np.arange(n)
+            s = O.index_scores(qi64[i], ic64, ids)
+            iou, _ = topk_row_check(idx[b, i], s, ids, k, acc_bound(qi64[i], ic64[:n]), f"b{b} t{t}")
+            ious.append(iou)
+    assert np.mean(ious) >= 0.999
+
+
+@pytest.mark.parametrize("dtype,B,T,nc,dI,blk,m,k", [
+    ("f32", 1, 200, 300, 32, 16, 4, 20),
+    ("bf16", 2, 400, 5000, 128, 128, 8, 256),
+    ("bf16", 1, 64, 32768, 128, 128, 64, 2048),
+])
+def test_index_hisa(S, dtype, B, T, nc, dI, blk, m, k):
+    r = 4
+    sc = 1.0 if dtype == "f32" else dI ** -0.5
+    ic = _normal("ic", (B, nc, dI), sc, dtype)
+    qi = _normal("qi", (B, T, dI), sc, dtype)
+    q_pos = _positions(B, T, r * nc + 40, 6)
+    icd, qid, qpd = ic.to(dev), qi.to(dev), q_pos.to(dev)
+    reps = S.layer.block_reps(icd, nc, blk)
+    idx = S.layer.index_topk(qid, qpd, icd, nc, r, k, S.HYB_INDEX_HISA, reps, blk, m, 128)
+    # with every block kept, HISA must reproduce the flat indexer exactly
+    idx_all = S.layer.index_topk(qid, qpd, icd, nc, r, k, S.HYB_INDEX_HISA, reps, blk, nc // blk + 1, 0)
+    idx_flat = S.layer.index_topk(qid, qpd, icd, nc, r, k)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_all, idx_flat)
+    idx = idx.cpu().numpy()
+    exact_rows = 0
+    for b in range(B):
+        ic64, qi64 = to64(ic[b]), to64(qi[b])
+        reps64 = O.block_reps(ic64, blk, dtype)
+        for i in range(T):
+            t = int(q_pos[b, i])
+            n = O.visible_entries(t, r, nc)
+            full = n // blk
+            m_full = m - (1 if n % blk else 0)
+            # stage-1 near ties (blocks) may legitimately pick other blocks: skip those rows
+            if 0 < m_full < full:
+                bs = reps64[:full] @ qi64[i]
+                srt = np.sort(bs)[::-1]
+                if srt[m_full - 1] - srt[m_full] <= 1e-3 * max(abs(srt[m_full - 1]), abs(srt[m_full])):
+                    continue
+            blocks = O.hisa_blocks(qi64[i], reps64, n, blk, m)
+            ids = np.concatenate([np.arange(g * blk, min((g + 1) * blk, n)) for g in blocks]) \
+                if len(blocks) else np.empty(0, dtype=np.int64)
+            s = O.index_scores(qi64[i], ic64, ids)
+            topk_row_check(idx[b, i], s, ids, k, acc_bound(qi64[i], ic64[ids]), f"hisa b{b} t{t}")
+            exact_rows += 1
+    assert exact_rows >= 0.9 * B * T
+
+
+# --------------------------------------------------------------------------- S3
+
+
+def _random_sel(B, T, k, q_pos, r, nc, seed):
+    """Random distinct visible entries per query (ascending), -1 padded: an input
+    for testing attention on its own."""
+    out = np.full((B, T, k), -1, dtype=np.int32)
+    for b in range(B):
+        for i in range(T):
+            n = O.visible_entries(int(q_pos[b, i]), r, nc)
+            if n == 0:
+                continue
+            keys = rng.raw_u64(seed, f"sel_{b}_{i}", 0, n)
+            pick = np.sort(torch.argsort(keys)[:min(k, n)].numpy())
+            cut = min(len(pick), k - (i % 3))           # some rows shorter than k
+            out[b, i, :cut] = pick[:cut]
+    return torch.from_numpy(out)
+
+
+@pytest.mark.parametrize("dtype,B,T,H,D,nc,r,k,W,L,mode", [
+    ("f32", 1, 120, 8, 64, 128, 4, 16, 32, 512, "prefill"),
+    ("f32", 1, 120, 8, 64, 4, 128, 0, 32, 512, "prefill"),
+    ("bf16", 2, 150, 64, 128, 2000, 4, 96, 128, 8000, "prefill"),
+    ("bf16", 2, 150, 64, 128, 60, 128, 0, 128, 7680, "prefill"),
+    ("bf16", 2, 150, 64, 128, 2000, 4, 96, 128, 8000, "decode"),
+    ("bf16", 3, 2, 64, 128, 60, 128, 0, 128, 7680, "decode"),
+])
+def test_attention(S, dtype, B, T, H, D, nc, r, k, W, L, mode):
+    sc = 1.0 if dtype == "f32" else D ** -0.5
+    q = _normal("q", (B, T, H, D), sc, dtype)
+    kc, vc = _normal("kc", (B, nc, D), sc, dtype), _normal("vc", (B, nc, D), sc, dtype)
+    kw, vw = _normal("kw", (B, L, D), sc, dtype), _normal("vw", (B, L, D), sc, dtype)
+    q_pos = _positions(B, T, L, 7)
+    idx = _random_sel(B, T, k, q_pos, r, nc, 8) if k > 0 else None
+    md = S.HYB_ATTN_PREFILL if mode == "prefill" else S.HYB_ATTN_DECODE
+    scale = 1.0 / math.sqrt(D)
+    g = lambda t: None if t is None else t.to(dev)
+    o, lse = S.layer.attention(g(q), g(q_pos), g(kc), g(vc), nc, r, g(idx), g(kw), g(vw), W, scale, md)
+    torch.cuda.synchronize()
+    kind = "csa" if k > 0 else "hca"
+    p = O.LayerParams(kind, r, kind == "csa", W, scale, dtype, k=k)
+    want_o, want_l = [], []
+    for b in range(B):
+        kc64, vc64, kw64, vw64 = to64(kc[b]), to64(vc[b]), to64(kw[b]), to64(vw[b])
+        for i in range(T):
+            t = int(q_pos[b, i])
+            n = O.visible_entries(t, r, nc)
+            sel = idx[b, i].numpy() if k > 0 else np.arange(n)
+            keys, vals = O.key_set(t, sel[sel >= 0], kc64, vc64, kw64, vw64, L, W)
+            oo, ll = O.attend(to64(q[b, i]), keys, vals, scale)
+            want_o.append(O.round_store(oo, dtype))
+            want_l.append(ll)
+    check_close(to64(o).reshape(B * T, H, D), np.stack(want_o), dtype, f"attention {mode}")
+    np.testing.assert_allclose(to64(lse).reshape(B * T, H), np.stack(want_l), rtol=0,
+                               atol=1e-4 if dtype == "f32" else 1e-3)
+
+
+def test_attention_reports_bad_index(S):
+    B, T, H, D, nc, k, W, L = 1, 4, 64, 128, 100, 8, 128, 600
+    q = _normal("q", (B, T, H, D), 0.1, "bf16").to(dev)
+    kc = _normal("kc", (B, nc, D), 0.1, "bf16").to(dev)
+    kw = _normal("kw", (B, L, D), 0.1, "bf16").to(dev)
+    q_pos = torch.full((B, T), 500, dtype=torch.int32, device=dev)
+    idx = torch.arange(k, dtype=torch.int32, device=dev).repeat(B, T, 1).contiguous()
+    idx[0, 2, 3] = 10 ** 6                                   # out of range: skipped and reported
+    S.layer.attention(q, q_pos, kc, kc, nc, 4, idx, kw, kw, W, 0.1)
+    assert S.abi.hyb_get_device_status() == S.abi.HYB_ERR_DEVICE_CHECK
