@@ -9,7 +9,11 @@
 #include "compress.cuh"
 #include "topk.cuh"
 #include "index.cuh"
+#include "index_tc.cuh"
 #include "attn.cuh"
+#include "attn_tc.cuh"
+
+#include <type_traits>
 
 using namespace hyb;
 
@@ -75,6 +79,22 @@ cudaError_t allow_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+// Scores of query rows [i0, i0+nq) against keys (entries or block representatives):
+// tensor cores for bf16 when the shape allows, CUDA cores otherwise.
+template <typename T>
+cudaError_t launch_scores(const void* qi, const int* q_pos, const void* keys, float* S, int batch, int T_, int i0,
+                          int nq, int dI, int keys_cap, int r, int nc, int div, int ldS, cudaStream_t stream) {
+  const int max_cols = nc / div;
+  if (max_cols <= 0) return cudaSuccess;
+  if (std::is_same<T, bf16>::value && tc_scores_supported(dI, qi, keys))
+    return launch_scores_tc(qi, q_pos, keys, S, batch, T_, i0, nq, dI, keys_cap, r, nc, div, ldS, max_cols, stream);
+  dim3 g((max_cols + kSB_N - 1) / kSB_N, (nq + kSB_M - 1) / kSB_M, batch);
+  scores_ffma_kernel<T><<<g, 256, 0, stream>>>((const T*)qi, q_pos, (const T*)keys, S, T_, i0, nq, dI, keys_cap,
+                                               r, nc, div, ldS);
+  count_launch();
+  return cudaGetLastError();
+}
+
 template <typename T>
 int index_topk_impl(int batch, int T_, int dI, const void* qi, const int* q_pos, const void* ic,
                     int nc, int nc_cap, int r, int k, int mode, const void* reps, int nb_cap,
@@ -85,12 +105,9 @@ int index_topk_impl(int batch, int T_, int dI, const void* qi, const int* q_pos,
   for (int i0 = 0; i0 < T_; i0 += p.nq) {
     const int nq = T_ - i0 < p.nq ? T_ - i0 : p.nq;
     if (mode == HYB_INDEX_FLAT) {
-      dim3 g((nc + kSB_N - 1) / kSB_N, (nq + kSB_M - 1) / kSB_M, batch);
-      if (nc > 0) {
-        scores_ffma_kernel<T><<<g, 256, 0, stream>>>((const T*)qi, q_pos, (const T*)ic, S, T_, i0, nq,
-                                                     dI, nc_cap, r, nc, 1, p.ldS);
-        count_launch();
-      }
+      if ((e = launch_scores<T>(qi, q_pos, ic, S, batch, T_, i0, nq, dI, nc_cap, r, nc, 1, p.ldS, stream)) !=
+          cudaSuccess)
+        return HYB_ERR_CUDA;
       const size_t smem = p.global_keys ? 0 : (size_t)nc * 4;
       if ((e = allow_smem(select_flat_kernel, smem)) != cudaSuccess) return HYB_ERR_CUDA;
       uint32_t* gkeys = p.global_keys ? reinterpret_cast<uint32_t*>(ws + p.off_keys) : nullptr;
@@ -267,7 +284,8 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const
     return HYB_ERR_INVALID_ARG;
   if (batch == 0 || T == 0) return HYB_OK;
   if (!q || !q_pos || !kw || !vw || !o || ((nc > 0) && (!kc || !vc))) return HYB_ERR_INVALID_ARG;
-  if (!attn_ffma_supported(H, D)) return HYB_ERR_UNSUPPORTED;
+  if (!attn_ffma_supported(H, D) && !(dtype == HYB_DTYPE_BF16 && attn_tc_supported(H, D, q, kc, vc, kw, vw)))
+    return HYB_ERR_UNSUPPORTED;
   const int n_keys = (idx ? k : nc) + W;
   const int ns = attn_splits(mode, batch, T, n_keys);
   AttnArgs a{q, q_pos, kc, vc, nc, nc_cap, r, idx, k, kw, vw, ring, W, scale, o, lse,
@@ -285,7 +303,11 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const
     if ((e = launch_attn_ffma<float>(a, batch, s)) != cudaSuccess) return HYB_ERR_CUDA;
     if (ns > 1) { attn_merge_kernel<float><<<dim3(batch * T, H), 128, 0, s>>>(a); count_launch(); }
   } else {
-    if ((e = launch_attn_ffma<bf16>(a, batch, s)) != cudaSuccess) return HYB_ERR_CUDA;
+    if (attn_tc_supported(H, D, q, kc, vc, kw, vw))
+      e = launch_attn_tc(a, batch, s);
+    else
+      e = launch_attn_ffma<bf16>(a, batch, s);
+    if (e != cudaSuccess) return HYB_ERR_CUDA;
     if (ns > 1) { attn_merge_kernel<bf16><<<dim3(batch * T, H), 128, 0, s>>>(a); count_launch(); }
   }
   return cuda_status(cudaGetLastError());

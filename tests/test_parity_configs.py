@@ -93,8 +93,9 @@ def _compare_rows(w, ly, p, gpu, b, rows, q, qi, q_pos, caches, ring_k, ring_v, 
             iou, _ = topk_row_check(gidx[gi], s, ids, ly.k, eps, f"{w.name} row {i}")
             ious.append(iou)
             same = set(gidx[gi][gidx[gi] >= 0].tolist()) == set(idx[idx >= 0].tolist())
-            for j in planted:
-                if j < n_vis and np.dot(qi[i], ic[j]) > 0.4 * np.linalg.norm(qi[i]) * np.linalg.norm(ic[j]):
+            for j in planted:   # the flat indexer must find every planted key a row can see
+                if ly.index_mode == "flat" and j < n_vis and \
+                        np.dot(qi[i], ic[j]) > 0.4 * np.linalg.norm(qi[i]) * np.linalg.norm(ic[j]):
                     assert j in set(gidx[gi].tolist()), f"planted entry {j} missed by row {i}"
         allp.append((go[gi], o))
         if same:

@@ -72,8 +72,9 @@ def test_compress(S, dtype, B, L, D, dI, r, overlap, j0, j1):
         for gt, wt, nm in zip(got, want, "kvi"):
             g64 = to64(gt)
             check_close(g64, wt, dtype, f"compress {nm} b={b}")
-            if dtype == "bf16":   # at most one bf16 ulp from the fp64 result rounded once
-                assert np.all(np.abs(g64 - wt) <= _ulp_bf16(wt) * 1.0001), f"{nm}: more than one ulp"
+            if dtype == "bf16":   # one bf16 ulp from the fp64 result, plus the fp32 accumulation error
+                slack = 2.0 ** -20 * max(1.0, float(np.abs(wt).max()))
+                assert np.all(np.abs(g64 - wt) <= _ulp_bf16(wt) * 1.0001 + slack), f"{nm}: more than one ulp"
         assert torch.all(kc[b, :j0] == 0) and torch.all(kc[b, j1:] == 0)   # nothing outside the range
 
 
@@ -86,7 +87,7 @@ def test_block_reps(S):
     for b in range(B):
         want = O.block_reps(to64(ic[b]), blk, "bf16")
         got = to64(reps[b, :nc // blk])
-        assert np.all(np.abs(got - want) <= _ulp_bf16(want) * 1.0001)
+        assert np.all(np.abs(got - want) <= _ulp_bf16(want) * 1.0001 + 2.0 ** -20)
     assert torch.all(reps[:, nc // blk:] == 0)
 
 
@@ -107,6 +108,8 @@ def _positions(B, T, hi, seed):
     ("bf16", 2, 700, 3000, 128, 4, 64, 128),
     ("bf16", 64, 1, 8192, 128, 4, 512, 0),
     ("bf16", 1, 200, 33000, 128, 4, 2048, 0),
+    ("bf16", 2, 300, 2000, 64, 4, 64, 0),      # tensor-core scorer, one 64-wide K block
+    ("bf16", 2, 300, 1000, 96, 4, 32, 0),      # CUDA-core scorer (width not built for tensor cores)
 ])
 def test_index_flat(S, dtype, B, T, nc, dI, r, k, chunk):
     sc = 1.0 if dtype == "f32" else dI ** -0.5
