@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU oracle sample")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-only", action="store_true", help="time only the prefill step (profiling runs)")
+    ap.add_argument("--L", type=int, default=None, help="override the prefill length (profiling runs)")
     return ap.parse_args()
 
 
@@ -398,7 +400,7 @@ def run_reference(args, world, rank):
 def run_ours(args, world, rank, local):
     import sparse_attention_hyb_b200 as S
     S.abi.lib()
-    w = C.PREFILL_32K
+    w = C.PREFILL_32K if args.L is None else C.scaled(C.PREFILL_32K, L=args.L, T=args.L)
     pk, pk_src = peaks()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     clock = ClockSampler(local)
@@ -411,8 +413,12 @@ def run_ours(args, world, rank, local):
     achieved = res["attn_flops"] / (attn_ms / 1e3) / 1e12
     peak = pk["bf16_tflops"]
     traffic = measured_traffic("attention")
-    e2e_ms, h2d, d2h = bench_e2e(S, st, max(3, args.steps // 2))
-    e2e_ms = max_over_ranks(e2e_ms, world)
+    if args.prefill_only:
+        args.no_decode = args.no_cpu_baseline = True
+        e2e_ms, h2d, d2h = float("nan"), 0, 0
+    else:
+        e2e_ms, h2d, d2h = bench_e2e(S, st, max(3, args.steps // 2))
+        e2e_ms = max_over_ranks(e2e_ms, world)
     decode = None if args.no_decode else bench_decode(S, args.steps, args.warmup, flush)
     if S.abi.hyb_get_device_status() != 0:
         raise RuntimeError("device status error after the benchmark")

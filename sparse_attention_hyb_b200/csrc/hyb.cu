@@ -10,6 +10,7 @@
 #include "topk.cuh"
 #include "index.cuh"
 #include "index_tc.cuh"
+#include "topk_reg.cuh"
 #include "attn.cuh"
 #include "attn_tc.cuh"
 
@@ -108,11 +109,18 @@ int index_topk_impl(int batch, int T_, int dI, const void* qi, const int* q_pos,
       if ((e = launch_scores<T>(qi, q_pos, ic, S, batch, T_, i0, nq, dI, nc_cap, r, nc, 1, p.ldS, stream)) !=
           cudaSuccess)
         return HYB_ERR_CUDA;
-      const size_t smem = p.global_keys ? 0 : (size_t)nc * 4;
-      if ((e = allow_smem(select_flat_kernel, smem)) != cudaSuccess) return HYB_ERR_CUDA;
-      uint32_t* gkeys = p.global_keys ? reinterpret_cast<uint32_t*>(ws + p.off_keys) : nullptr;
-      select_flat_kernel<<<dim3(nq, batch), kTopkThreads, smem, stream>>>(S, q_pos, idx, T_, i0, nq, r,
-                                                                          nc, k, p.ldS, gkeys);
+      if (nc <= 256 * kRegEPT) {
+        select_flat_reg_kernel<256><<<dim3(nq, batch), 256, 0, stream>>>(S, q_pos, idx, T_, i0, nq, r, nc, k, p.ldS);
+      } else if (nc <= 1024 * kRegEPT) {
+        select_flat_reg_kernel<1024><<<dim3(nq, batch), 1024, 0, stream>>>(S, q_pos, idx, T_, i0, nq, r, nc, k,
+                                                                           p.ldS);
+      } else {
+        const size_t smem = p.global_keys ? 0 : (size_t)nc * 4;
+        if ((e = allow_smem(select_flat_kernel, smem)) != cudaSuccess) return HYB_ERR_CUDA;
+        uint32_t* gkeys = p.global_keys ? reinterpret_cast<uint32_t*>(ws + p.off_keys) : nullptr;
+        select_flat_kernel<<<dim3(nq, batch), kTopkThreads, smem, stream>>>(S, q_pos, idx, T_, i0, nq, r,
+                                                                            nc, k, p.ldS, gkeys);
+      }
       count_launch();
     } else {
       int* blk = reinterpret_cast<int*>(ws + p.off_blk);
@@ -124,18 +132,35 @@ int index_topk_impl(int batch, int T_, int dI, const void* qi, const int* q_pos,
                                                      dI, nb_cap, r, nc, block, p.ldS);
       count_launch();
       }
-      const size_t smem1 = (size_t)(p.nb > 0 ? p.nb : 1) * 4;
-      if ((e = allow_smem(select_blocks_kernel, smem1)) != cudaSuccess) return HYB_ERR_CUDA;
-      select_blocks_kernel<<<dim3(nq, batch), kTopkThreads, smem1, stream>>>(S, q_pos, blk, T_, i0, nq, r,
-                                                                             nc, block, top_m, p.ldS);
+      if (p.nb <= 256 * kRegEPT) {
+        select_blocks_reg_kernel<256><<<dim3(nq, batch), 256, 0, stream>>>(S, q_pos, blk, T_, i0, nq, r, nc, block,
+                                                                          top_m, p.ldS);
+      } else if (p.nb <= 1024 * kRegEPT) {
+        select_blocks_reg_kernel<1024><<<dim3(nq, batch), 1024, 0, stream>>>(S, q_pos, blk, T_, i0, nq, r, nc,
+                                                                            block, top_m, p.ldS);
+      } else {
+        const size_t smem1 = (size_t)(p.nb > 0 ? p.nb : 1) * 4;
+        if ((e = allow_smem(select_blocks_kernel, smem1)) != cudaSuccess) return HYB_ERR_CUDA;
+        select_blocks_kernel<<<dim3(nq, batch), kTopkThreads, smem1, stream>>>(S, q_pos, blk, T_, i0, nq, r,
+                                                                               nc, block, top_m, p.ldS);
+      }
       count_launch();
       hisa_cand_scores_kernel<T><<<dim3(nq, batch), 256, dI * 4, stream>>>(
           (const T*)qi, q_pos, (const T*)ic, blk, SC, ncand, T_, i0, nq, dI, nc_cap, r, nc, block, top_m);
       count_launch();
-      const size_t smem2 = (size_t)top_m * block * 4;
-      if ((e = allow_smem(select_cand_kernel, smem2)) != cudaSuccess) return HYB_ERR_CUDA;
-      select_cand_kernel<<<dim3(nq, batch), kTopkThreads, smem2, stream>>>(SC, ncand, blk, idx, T_, i0, nq,
-                                                                           block, top_m, k);
+      const int n2 = top_m * block;
+      if (n2 <= 256 * kRegEPT) {
+        select_cand_reg_kernel<256><<<dim3(nq, batch), 256, 0, stream>>>(SC, ncand, blk, idx, T_, i0, nq, block,
+                                                                        top_m, k);
+      } else if (n2 <= 1024 * kRegEPT) {
+        select_cand_reg_kernel<1024><<<dim3(nq, batch), 1024, 0, stream>>>(SC, ncand, blk, idx, T_, i0, nq, block,
+                                                                          top_m, k);
+      } else {
+        const size_t smem2 = (size_t)n2 * 4;
+        if ((e = allow_smem(select_cand_kernel, smem2)) != cudaSuccess) return HYB_ERR_CUDA;
+        select_cand_kernel<<<dim3(nq, batch), kTopkThreads, smem2, stream>>>(SC, ncand, blk, idx, T_, i0, nq,
+                                                                             block, top_m, k);
+      }
       count_launch();
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return HYB_ERR_CUDA;

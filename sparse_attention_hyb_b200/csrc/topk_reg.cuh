@@ -1,0 +1,217 @@
+// Top-k selection, register-resident variant (HISA write-up, section 01: keep
+// the k highest-scoring entries; ties go to the lower index).
+//
+// One CTA per row, each thread holding EPT consecutive scores of the row in
+// registers as order-preserving uint32 keys (blocked layout: thread t owns
+// positions [t*EPT, (t+1)*EPT)).  The k-th largest key K* is found exactly
+// with three radix passes of 11, 11 and 10 bits.  The first pass, where most
+// keys share a few high digits, counts into 8 privatised histograms (two
+// 16-bit counters per word) that are summed afterwards; later passes only see
+// the keys that still match the prefix.  Because the layout is blocked, the
+// ordered output needs a single block-wide exclusive scan of per-thread
+// (greater-than, equal-to) counts; every thread then writes its selected
+// positions in ascending order, the lowest-index keys equal to K* first.
+#pragma once
+#include "common.cuh"
+#include "topk.cuh"
+
+namespace hyb {
+
+constexpr int kRegEPT = 32;
+
+template <int THREADS>
+struct RegSelSmem {
+  uint32_t hist_w[8][1024];
+  uint32_t hist[2048];
+  uint32_t warp_tot[THREADS / 32];
+  uint32_t warp_off[THREADS / 32];
+  uint32_t total;
+  uint32_t prefix, remaining;
+};
+
+// Exclusive prefix sum over the CTA of one value per thread; `total` receives the sum.
+template <int THREADS>
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, RegSelSmem<THREADS>& sh, uint32_t& total) {
+  constexpr int NW = THREADS / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) sh.warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t t = lane < NW ? sh.warp_tot[lane] : 0u;
+    uint32_t ti = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t u = __shfl_up_sync(0xffffffffu, ti, o);
+      if (lane >= o) ti += u;
+    }
+    if (lane < NW) sh.warp_off[lane] = ti - t;
+    if (lane == 31) sh.total = ti;
+  }
+  __syncthreads();
+  total = sh.total;
+  return sh.warp_off[warp] + incl - v;
+}
+
+// Finds the digit d (bins of width 2048 / THREADS per thread) such that
+// above(d) < rem <= above(d) + hist[d]; stores prefix |= d << shift, remaining.
+template <int THREADS>
+__device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift) {
+  constexpr int BPT = 2048 / THREADS;
+  uint32_t h[BPT], tot = 0;
+#pragma unroll
+  for (int e = 0; e < BPT; ++e) { h[e] = sh.hist[threadIdx.x * BPT + e]; tot += h[e]; }
+  const uint32_t rem = sh.remaining;
+  const uint32_t prefix = sh.prefix;
+  uint32_t total;
+  const uint32_t before = block_exclusive_scan<THREADS>(tot, sh, total);
+  uint32_t above = total - before - tot;    // keys in bins above this thread's range
+  if (above < rem && rem <= above + tot) {
+#pragma unroll
+    for (int e = BPT - 1; e >= 0; --e) {
+      if (above + h[e] >= rem) {
+        sh.prefix = prefix | ((uint32_t)(threadIdx.x * BPT + e) << shift);
+        sh.remaining = rem - above;
+        break;
+      }
+      above += h[e];
+    }
+  }
+  __syncthreads();
+}
+
+template <int THREADS, typename Map>
+__device__ void select_row_reg(const float* __restrict__ scores, int n, int k, int k_out, int* __restrict__ out,
+                               Map map, RegSelSmem<THREADS>& sh) {
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (n <= k) {
+    for (int i = tid; i < k_out; i += THREADS) out[i] = i < n ? map(i) : -1;
+    return;
+  }
+  for (int i = k + tid; i < k_out; i += THREADS) out[i] = -1;
+  const int base = tid * kRegEPT;
+  const int cnt = n - base < 0 ? 0 : (n - base > kRegEPT ? kRegEPT : n - base);
+  uint32_t key[kRegEPT];
+  if (cnt == kRegEPT && (reinterpret_cast<uintptr_t>(scores + base) & 15) == 0) {
+#pragma unroll
+    for (int e = 0; e < kRegEPT; e += 4) {
+      const float4 f = *reinterpret_cast<const float4*>(scores + base + e);
+      key[e] = score_key(f.x); key[e + 1] = score_key(f.y); key[e + 2] = score_key(f.z); key[e + 3] = score_key(f.w);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kRegEPT; ++e) key[e] = e < cnt ? score_key(scores[base + e]) : 0u;
+  }
+  // ---- pass 0: bits 31..21, privatised histograms
+  for (int i = tid; i < 8 * 1024; i += THREADS) (&sh.hist_w[0][0])[i] = 0u;
+  if (tid == 0) { sh.prefix = 0; sh.remaining = (uint32_t)k; }
+  __syncthreads();
+  uint32_t* hw = sh.hist_w[warp & 7];
+#pragma unroll
+  for (int e = 0; e < kRegEPT; ++e)
+    if (e < cnt) {
+      const uint32_t d = key[e] >> 21;
+      atomicAdd(&hw[d >> 1], 1u << ((d & 1) * 16));
+    }
+  __syncthreads();
+  for (int b = tid; b < 2048; b += THREADS) {
+    uint32_t s = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += (sh.hist_w[w][b >> 1] >> ((b & 1) * 16)) & 0xFFFFu;
+    sh.hist[b] = s;
+  }
+  __syncthreads();
+  find_digit<THREADS>(sh, 21);
+  // ---- passes 1, 2: bits 20..10 and 9..0 of the keys that match the prefix
+  uint32_t mask = 0xFFE00000u;
+#pragma unroll 1
+  for (int pass = 1; pass < 3; ++pass) {
+    const int shift = pass == 1 ? 10 : 0;
+    const uint32_t dmask = pass == 1 ? 0x7FFu : 0x3FFu;
+    for (int b = tid; b < 2048; b += THREADS) sh.hist[b] = 0u;
+    __syncthreads();
+    const uint32_t prefix = sh.prefix;
+#pragma unroll
+    for (int e = 0; e < kRegEPT; ++e)
+      if (e < cnt && (key[e] & mask) == prefix) atomicAdd(&sh.hist[(key[e] >> shift) & dmask], 1u);
+    __syncthreads();
+    find_digit<THREADS>(sh, shift);
+    mask |= dmask << shift;
+  }
+  const uint32_t kth = sh.prefix, need = sh.remaining;
+  // ---- ordered output
+  uint32_t gt = 0, eq = 0;
+#pragma unroll
+  for (int e = 0; e < kRegEPT; ++e)
+    if (e < cnt) { gt += key[e] > kth; eq += key[e] == kth; }
+  uint32_t total;
+  const uint32_t before = block_exclusive_scan<THREADS>((gt << 16) | eq, sh, total);
+  uint32_t gt_run = before >> 16, eq_run = before & 0xFFFFu;
+#pragma unroll
+  for (int e = 0; e < kRegEPT; ++e) {
+    if (e >= cnt) break;
+    const uint32_t kv = key[e];
+    if (kv > kth) {
+      out[gt_run + (eq_run < need ? eq_run : need)] = map(base + e);
+      ++gt_run;
+    } else if (kv == kth) {
+      if (eq_run < need) out[gt_run + eq_run] = map(base + e);
+      ++eq_run;
+    }
+  }
+}
+
+// Flat rows: row (b, i) keeps the k best of its visible entries.
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS)
+select_flat_reg_kernel(const float* __restrict__ S, const int* __restrict__ q_pos, int* __restrict__ idx, int T_,
+                       int i0, int nq, int r, int nc, int k, int ldS) {
+  __shared__ RegSelSmem<THREADS> sh;
+  const int b = blockIdx.y, m = blockIdx.x;
+  const size_t row = (size_t)b * T_ + i0 + m;
+  const int n = visible_entries(q_pos[row], r, nc);
+  select_row_reg<THREADS>(S + ((size_t)b * nq + m) * ldS, n, k, k, idx + row * k, IdentityMap{}, sh);
+}
+
+// HISA stage 1: the partial block (if any) is always kept; the best full blocks
+// fill the other slots.  blk row: kept blocks ascending, then -1.
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS)
+select_blocks_reg_kernel(const float* __restrict__ SB, const int* __restrict__ q_pos, int* __restrict__ blk, int T_,
+                         int i0, int nq, int r, int nc, int block, int top_m, int ldB) {
+  __shared__ RegSelSmem<THREADS> sh;
+  const int b = blockIdx.y, m = blockIdx.x;
+  const size_t row = (size_t)b * T_ + i0 + m;
+  const int v = visible_entries(q_pos[row], r, nc);
+  const int full = v / block;
+  const bool partial = (v % block) != 0;
+  const int k1 = top_m - (partial ? 1 : 0);
+  int* out = blk + ((size_t)b * nq + m) * top_m;
+  if (k1 > 0) {
+    select_row_reg<THREADS>(SB + ((size_t)b * nq + m) * ldB, full, k1, top_m, out, IdentityMap{}, sh);
+  } else {
+    for (int i = threadIdx.x; i < top_m; i += THREADS) out[i] = -1;
+  }
+  __syncthreads();
+  if (partial && threadIdx.x == 0) out[full < k1 ? full : k1] = full;
+}
+
+// HISA stage 2: the k best candidates; candidate p is entry blocks[p / B] * B + p % B.
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS)
+select_cand_reg_kernel(const float* __restrict__ SC, const int* __restrict__ n_cand, const int* __restrict__ blk,
+                       int* __restrict__ idx, int T_, int i0, int nq, int block, int top_m, int k) {
+  __shared__ RegSelSmem<THREADS> sh;
+  const int b = blockIdx.y, m = blockIdx.x;
+  const size_t row = (size_t)b * T_ + i0 + m;
+  const size_t slot = (size_t)b * nq + m;
+  select_row_reg<THREADS>(SC + slot * ((size_t)top_m * block), n_cand[slot], k, k, idx + row * k,
+                          BlockListMap{blk + slot * top_m, block}, sh);
+}
+
+}  // namespace hyb
