@@ -143,6 +143,30 @@ int hyb_index_topk(int dtype, int batch, int T, int dI,
                    int* idx, void* ws, size_t ws_bytes, hyb_stream_t stream);
 
 /*
+ * Flat indexer with no caller-provided scratch (no counterpart on the pages:
+ * this is an interface for callers, not part of the method).
+ *
+ * Same arguments and results as hyb_index_topk in HYB_INDEX_FLAT mode, minus
+ * the workspace.  It is for callers that cannot allocate device memory for the
+ * library, such as an inference engine whose pool allocator owns all of HBM or
+ * a plugin whose host framework does every device allocation itself.  The
+ * library allocates nothing here either: the scores go to a 16 MiB array that
+ * is part of the library's device image, so every GPU that loads libhyb holds
+ * those 16 MiB until the process exits.
+ *  - The first call on a device (with that device current) looks up the
+ *    array's device address; make that first call before any stream capture.
+ *  - All calls on a device share the array.  Calls whose kernels may run at the
+ *    same time on that device (different streams without ordering) race on it
+ *    and must not be issued.
+ *  - Returns HYB_ERR_UNSUPPORTED when batch * round_up(nc, 4) * 4 bytes exceed
+ *    the 16 MiB array or nc > 32768; queries are scored in chunks that fit.
+ */
+int hyb_index_topk_noalloc(int dtype, int batch, int T, int dI,
+                           const void* qi, const int* q_pos,
+                           const void* ic, int nc, int nc_cap, int r, int k,
+                           int* idx, hyb_stream_t stream);
+
+/*
  * S3 + S4 — shared-KV attention with a sliding window (HCA article, section
  * "怎么压": MQA over all compressed entries (HCA) plus a 128-token window branch,
  * as in CSA; trdm.cn 2.1: CSA attends the indexer's top-k plus the window).

@@ -39,6 +39,8 @@ SIGNATURES = {
     "hyb_index_topk": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int,
                                 _c_int, _c_int, _c_int, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_ptr,
                                 _c_ptr, _c_size, _c_ptr]),
+    "hyb_index_topk_noalloc": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int,
+                                        _c_int, _c_int, _c_ptr, _c_ptr]),
     "hyb_attn_fwd_workspace_size": (_c_size, [_c_int] * 9),
     "hyb_attn_fwd": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_ptr, _c_ptr, _c_ptr, _c_ptr,
                               _c_int, _c_int, _c_int, _c_ptr, _c_int, _c_ptr, _c_ptr, _c_int, _c_int,
@@ -146,6 +148,14 @@ def hyb_index_topk(qi, q_pos, ic, nc: int, r: int, k: int, mode: int, reps, bloc
                               r, k, mode, _ptr(reps), reps.shape[1] if reps is not None else 0, block,
                               top_m, q_chunk, _ptr(idx), _ptr(ws), ws_bytes, _stream(stream))
     _check("hyb_index_topk", st)
+
+
+def hyb_index_topk_noalloc(qi, q_pos, ic, nc: int, r: int, k: int, idx, stream=None):
+    """Flat indexer whose scratch is a fixed array inside libhyb (no workspace argument)."""
+    B, T, dI = qi.shape
+    st = lib().hyb_index_topk_noalloc(_dtype_code(qi), B, T, dI, _ptr(qi), _ptr(q_pos), _ptr(ic), nc, ic.shape[1],
+                                      r, k, _ptr(idx), _stream(stream))
+    _check("hyb_index_topk_noalloc", st)
 
 
 def hyb_attn_fwd_workspace_size(dtype: int, batch: int, T: int, H: int, D: int, k: int, nc: int, W: int,

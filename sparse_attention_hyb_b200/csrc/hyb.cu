@@ -339,3 +339,65 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Flat indexer without caller-provided scratch.
+//
+// Some callers cannot hand the library device memory: an inference engine that
+// gives the whole of HBM to its own pool allocator (cudaMalloc then fails, or
+// fragments the pool), or a plugin running inside a host framework that owns
+// all device allocations.  hyb_index_topk_noalloc serves them: its scores live
+// in the fixed array below, which every GPU that loads this library holds until
+// the process exits.  All calls on a device share it and it keeps the previous
+// call's contents; nothing in it needs to start at zero (every score is written
+// before it is read), but two calls whose kernels overlap on the GPU (different
+// streams, no ordering between them) race on it.
+constexpr size_t kNoAllocScratchBytes = 16u << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+
+// Device address of the scratch array on the current device, looked up once per
+// device (the host-side symbol is not a device address).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HYB_ERR_CUDA;
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return HYB_ERR_CUDA;
+    g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
+  return HYB_OK;
+}
+}  // namespace
+
+extern "C" int hyb_index_topk_noalloc(int dtype, int batch, int T, int dI, const void* qi, const int* q_pos,
+                                      const void* ic, int nc, int nc_cap, int r, int k, int* idx,
+                                      hyb_stream_t stream) {
+  if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
+  if (batch < 0 || T < 0 || dI <= 0 || nc < 0 || nc_cap < nc || r < 1 || k < 1) return HYB_ERR_INVALID_ARG;
+  if (batch == 0 || T == 0) return HYB_OK;
+  if (!qi || !q_pos || !ic || !idx) return HYB_ERR_INVALID_ARG;
+  if (dI % 4 != 0) return HYB_ERR_UNSUPPORTED;
+  // one row of scores per batch entry must fit, and rows must not need the
+  // global-memory key buffer of the longest-row path
+  const size_t row_bytes = (size_t)round_up(nc > 0 ? nc : 1, 4) * 4;
+  if (nc > 1024 * kRegEPT || row_bytes * (size_t)batch > kNoAllocScratchBytes) return HYB_ERR_UNSUPPORTED;
+  int nq = (int)(kNoAllocScratchBytes / (row_bytes * (size_t)batch));
+  if (nq > T) nq = T;
+  const IndexPlan p = plan_index(dtype, batch, T, nc, k, HYB_INDEX_FLAT, 0, 0, nq);
+  if (p.total > kNoAllocScratchBytes || p.global_keys) return HYB_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  const int st = noalloc_scratch(&ws);
+  if (st != HYB_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  return dtype == HYB_DTYPE_F32
+      ? index_topk_impl<float>(batch, T, dI, qi, q_pos, ic, nc, nc_cap, r, k, HYB_INDEX_FLAT, nullptr, 0, 0, 0, p,
+                               idx, w, s)
+      : index_topk_impl<bf16>(batch, T, dI, qi, q_pos, ic, nc, nc_cap, r, k, HYB_INDEX_FLAT, nullptr, 0, 0, 0, p,
+                              idx, w, s);
+}
