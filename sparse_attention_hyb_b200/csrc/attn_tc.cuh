@@ -2,27 +2,38 @@
 // 64 query heads over the selected / all compressed entries plus the sliding
 // window, one joint softmax (HCA article, section "怎么压"; trdm.cn 2.1).
 //
-// Transposed formulation, so that every MMA has M = 128 (full rate) although
-// a query has only 64 heads and, in CSA, its own key set:
-//   S^T[key, h] = K_tile[key, :] . Q[h, :]        M=128 keys,  N=64 heads, K=D
-//   O^T[d, h]  += V_tile^T[d, key] . P^T[key, h]  M=128 (=D),  N=64 heads, K=128 keys
-// The keys of a query are processed in groups of up to 6 tiles of 128.  The
-// group's S^T tiles stay in tensor memory (6 x 64 columns); the softmax warps
-// (one thread per key lane) take the exact per-head maximum over the group
-// (elementwise max, then a warp transpose-reduce and a 4-warp combine), rescale
-// the O^T accumulator in tensor memory when a later group raises the maximum,
-// then write P^T = exp2((s - m) * scale * log2 e) as a bf16 MN-major operand
-// in shared memory, one 128-byte row per key.  Row sums are accumulated per
-// thread and reduced across lanes once per query.
+// Transposed formulation, so that every MMA has M = 128 (full rate) although a
+// query has only 64 heads and, in CSA, its own key set:
+//   S^T[key, h] = K_tile[key, :] . Q[h, :]        M=128 keys, N=64 heads, K=D
+//   O^T[d, h]  += V_tile^T[d, key] . P^T[key, h]  M=128 (=D), N=64 heads, K=128 keys
+// A query's keys (compressed entries first, then window positions, each padded
+// to whole tiles of 128) are processed in groups of up to 3 tiles.
 //
-// Roles (192 threads, one CTA per SM, persistent over work items):
-//   warp 0      producer: Q by 2-D TMA; K and V tiles by TMA gather4 (4 rows
-//               per instruction, every lane issuing its own rows), compressed
-//               keys and window keys in separate tiles;
-//   warp 1      TMEM owner; one thread issues all MMAs and commits;
-//   warps 2..5  softmax + epilogue (TMEM lane quadrant = warp % 4).
-// A work item is a query or, for split-KV decode, a tile-aligned slice of its
-// key list; slices write a partial (o, lse) that attn_merge combines.
+// Roles (12 warps, one CTA per SM, persistent over work items):
+//   warp 3      key tables: turns each group's key list (indexer output or the
+//               dense range, then the window) into source rows in shared memory
+//               one group ahead, so no role waits on a global index load;
+//   warp 0      Q (2-D TMA, double-buffered) and K tiles (TMA gather4, 4 rows
+//               per instruction, every lane issuing its own rows);
+//   warp 2      V tiles (TMA gather4);
+//   warp 1      TMEM owner; one thread issues every MMA: S^T of group g+1 is
+//               issued before O^T of group g, so the tensor core computes the
+//               next group's scores while the softmax warps turn the current
+//               scores into probabilities;
+//   warps 4..11 softmax and epilogue: thread = key lane (TMEM lane quadrant =
+//               warp % 4), warps 4-7 own heads 0-31 and warps 8-11 heads 32-63.
+// Tensor memory: two S^T buffers (3 tiles x 64 columns) and two O^T
+// accumulators (64 columns), 512 columns in all.
+//
+// Softmax: per group, the per-head maximum over the group's keys (elementwise
+// max over the tiles, a warp transpose-reduce across key lanes, a 4-warp
+// combine).  The running maximum only moves when a group exceeds it by more
+// than 8 (base-2 exponent units), in which case O^T and the per-thread row sums
+// are rescaled; otherwise probabilities are taken against the stale maximum
+// (they stay below 2^8).  P^T is written as a bf16 MN-major operand in shared
+// memory, one 128-byte row per key.  Row sums are reduced across key lanes once
+// per query.  A work item is a query or, for split-KV decode, a tile-aligned
+// slice of its keys; slices write partial (o, lse) pairs that attn_merge combines.
 #pragma once
 #include "attn.cuh"
 #include "common.cuh"
@@ -33,14 +44,17 @@ namespace hyb {
 namespace attn_tc {
 
 constexpr int kH = 64, kD = 128, kTile = 128;
-constexpr int kGroup = 6;               // S^T tiles per group (6 x 64 TMEM columns)
-constexpr int kKSt = 3, kVSt = 2, kPSt = 2;
-constexpr int kThreads = 192;
-constexpr int kQBytes = kH * kD * 2;                 // 16 KB (two 64-column sub-tiles)
-constexpr int kKVBytes = kTile * kD * 2;             // 32 KB (two 64-column sub-tiles)
-constexpr int kPBytes = kTile * kH * 2;              // 16 KB
-constexpr int kSmem = kQBytes + kKSt * kKVBytes + kVSt * kKVBytes + kPSt * kPBytes + 1024;
-constexpr uint32_t kOCol = kGroup * kH;              // O^T accumulator columns [384, 448)
+constexpr int kGT = 3;                                  // tiles per group
+constexpr int kQSt = 2, kKSt = 2, kVSt = 2, kPSt = 2, kTbl = 4;
+constexpr int kThreads = 384;
+constexpr int kQBytes = kH * kD * 2;                    // 16 KB, two 64-column sub-tiles
+constexpr int kKVBytes = kTile * kD * 2;                // 32 KB, two 64-column sub-tiles
+constexpr int kPBytes = kTile * kH * 2;                 // 16 KB
+constexpr int kSmem = kQSt * kQBytes + kKSt * kKVBytes + kVSt * kKVBytes + kPSt * kPBytes + 1024;
+constexpr uint32_t kSCols = kGT * kH;                   // 192 columns per S^T buffer
+constexpr uint32_t kOCol = 2 * kSCols;                  // O^T buffers at 384 and 448
+constexpr float kRescaleThreshold = 8.f;                // base-2 units
+constexpr int kTblArrivals = 32 + 32 + 256;             // K producer, V producer, softmax lanes
 
 struct Maps {
   CUtensorMap q, kc, vc, kw, vw;
@@ -76,32 +90,34 @@ struct Item {
     if (tile_beg > tile_end) tile_beg = tile_end;
   }
   __device__ int n_tiles() const { return tile_end - tile_beg; }
-  __device__ int n_groups() const { return (n_tiles() + kGroup - 1) / kGroup; }
 };
 
-// Source of key v of a tile: compressed entry (is_win = false) or window slot.
-// Returns -1 for padding / invalid keys (their scores are masked).
-__device__ __forceinline__ int key_source(const AttnArgs& a, const KeyList& kl, int tile, int kk, bool& is_win,
-                                          bool check) {
+// Source of key kk of a tile: entry index (compressed) or ring slot (window);
+// -1 for padding / invalid keys.  Reports indices outside the visible range.
+__device__ __forceinline__ int key_source(const AttnArgs& a, const KeyList& kl, int tile, int kk) {
   if (tile < kl.comp_tiles) {
-    is_win = false;
     const int u = tile * kTile + kk;
     if (u >= kl.n_comp) return -1;
-    const int j = a.idx ? a.idx[(size_t)kl.row * a.k + u] : u;
+    const int j = a.idx ? __ldg(a.idx + (size_t)kl.row * a.k + u) : u;
     if (j < 0) return -1;
     if (j >= kl.vis) {
-      if (check) report(HYB_ERR_DEVICE_CHECK);
+      report(HYB_ERR_DEVICE_CHECK);
       return -1;
     }
     return j;
   }
-  is_win = true;
   const int u = (tile - kl.comp_tiles) * kTile + kk;
   if (u >= kl.n_win) return -1;
   return (kl.w0 + u) % a.ring;
 }
 
-__device__ __forceinline__ void named_sync_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+struct KeyTable {
+  int rows[kTbl][kGT * kTile];   // source row in the gather map, -1 = masked key
+  int safe[kTbl][kGT];           // a row inside the map for masked keys of the tile
+  int win[kTbl][kGT];            // 1 if the tile holds window keys
+};
+
+__device__ __forceinline__ void named_sync_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 template <int N>
 __device__ __forceinline__ void xmax_step(float* v, int lane, int mask) {
@@ -123,14 +139,14 @@ __device__ __forceinline__ void xsum_step(float* v, int lane, int mask) {
     v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
   }
 }
-// After these, v[0], v[1] of lane l hold heads 2l, 2l+1 reduced over the warp.
-__device__ __forceinline__ void warp_xmax64(float* v, int lane) {
-  xmax_step<64>(v, lane, 16); xmax_step<32>(v, lane, 8); xmax_step<16>(v, lane, 4);
-  xmax_step<8>(v, lane, 2); xmax_step<4>(v, lane, 1);
+// 32 values per lane -> v[0] of lane l holds element l reduced over the warp.
+__device__ __forceinline__ void warp_xmax32(float* v, int lane) {
+  xmax_step<32>(v, lane, 16); xmax_step<16>(v, lane, 8); xmax_step<8>(v, lane, 4);
+  xmax_step<4>(v, lane, 2); xmax_step<2>(v, lane, 1);
 }
-__device__ __forceinline__ void warp_xsum64(float* v, int lane) {
-  xsum_step<64>(v, lane, 16); xsum_step<32>(v, lane, 8); xsum_step<16>(v, lane, 4);
-  xsum_step<8>(v, lane, 2); xsum_step<4>(v, lane, 1);
+__device__ __forceinline__ void warp_xsum32(float* v, int lane) {
+  xsum_step<32>(v, lane, 16); xsum_step<16>(v, lane, 8); xsum_step<8>(v, lane, 4);
+  xsum_step<4>(v, lane, 2); xsum_step<2>(v, lane, 1);
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
@@ -148,6 +164,19 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2-slot ring helpers: use u of a slot -> phase parity.
+__device__ __forceinline__ uint32_t full_par(uint32_t n, int nst) { return (n / nst) & 1u; }
+__device__ __forceinline__ uint32_t empty_par(uint32_t n, int nst) { return ((n / nst) & 1u) ^ 1u; }
+
+struct PendingPV {
+  int valid, ob, ntiles, first;
+};
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
@@ -155,28 +184,32 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kQBytes;
+  uint8_t* sK = sQ + kQSt * kQBytes;
   uint8_t* sV = sK + kKSt * kKVBytes;
   uint8_t* sP = sV + kVSt * kKVBytes;
 
-  __shared__ uint64_t q_full, q_empty, k_full[kKSt], k_empty[kKSt], v_full[kVSt], v_empty[kVSt];
-  __shared__ uint64_t s_full[kGroup], s_free, p_full[kPSt], p_empty[kPSt], o_full, o_ready, mma_done;
+  __shared__ uint64_t q_full[kQSt], q_empty[kQSt], k_full[kKSt], k_empty[kKSt], v_full[kVSt], v_empty[kVSt];
+  __shared__ uint64_t s_full[2], s_free[2], p_full[kPSt], p_empty[kPSt], o_full[2], o_ready[2];
+  __shared__ uint64_t t_full[kTbl], t_empty[kTbl], mma_done;
+  __shared__ KeyTable tbl;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
-  __shared__ float red[4][kH];
-  __shared__ float m_run[kH], m_use[kH], alpha[kH], l_fin[kH];
+  __shared__ float red[2][4][32];
+  __shared__ float m_run[kH], m_use[kH], alpha_s[kH], l_fin[kH];
+  __shared__ int resc_flag[2];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     abort_flag = 0;
-    mbar_init(&q_full, 1); mbar_init(&q_empty, 1);
+    for (int s = 0; s < kQSt; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
     for (int s = 0; s < kKSt; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
     for (int s = 0; s < kVSt; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
-    for (int s = 0; s < kGroup; ++s) mbar_init(&s_full[s], 1);
-    mbar_init(&s_free, 4);
-    for (int s = 0; s < kPSt; ++s) { mbar_init(&p_full[s], 4); mbar_init(&p_empty[s], 1); }
-    mbar_init(&o_full, 1);
-    mbar_init(&o_ready, 4);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1); mbar_init(&s_free[s], 8);
+      mbar_init(&o_full[s], 1); mbar_init(&o_ready[s], 8);
+    }
+    for (int s = 0; s < kPSt; ++s) { mbar_init(&p_full[s], 8); mbar_init(&p_empty[s], 1); }
+    for (int s = 0; s < kTbl; ++s) { mbar_init(&t_full[s], 32); mbar_init(&t_empty[s], kTblArrivals); }
     mbar_init(&mma_done, 1);
     fence_mbar_init();
   }
@@ -187,306 +220,359 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   const uint32_t tmem = tmem_base;
   const float c2 = a.scale * 1.4426950408889634f;  // scale * log2(e)
 
-  if (warp == 0) {
-    // ======================================================== producer
-    uint32_t qn = 0, kn = 0, vn = 0;
-    if (lane == 0) { prefetch_tmap(&maps.q); prefetch_tmap(&maps.kc); prefetch_tmap(&maps.kw); }
+  // Register split per warpgroup.  Launch: 384 threads x 168 = 64512 registers;
+  // after the split 128 x 88 + 256 x 200 = 62464, within the launch's total.
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+  if (warp == 3) {
+    // ======================================================== key tables
+    uint32_t G = 0;
     for (int w = blockIdx.x; w < n_items && !abort_flag; w += gridDim.x) {
       Item it;
       it.init(a, w);
-      if (it.n_tiles() == 0) continue;
-      bool ok = true;
-      if (lane == 0) {
-        ok = mbar_wait(&q_empty, (qn & 1) ^ 1, &abort_flag);
-        if (ok) {
-          mbar_expect_tx(&q_full, kQBytes);
-          for (int c = 0; c < 2; ++c) tma_load_2d(sQ + c * (kQBytes / 2), &maps.q, &q_full, c * 64, it.kl.row * kH);
-        }
-      }
-      ++qn;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      for (int g0 = it.tile_beg; g0 < it.tile_end && ok; g0 += kGroup) {
-        const int g1 = min(it.tile_end, g0 + kGroup);
-        for (int pass = 0; pass < 2 && ok; ++pass) {  // K tiles of the group, then its V tiles
-          for (int tile = g0; tile < g1 && ok; ++tile) {
-            const int st = pass == 0 ? kn % kKSt : vn % kVSt;
-            const uint32_t ph = pass == 0 ? (kn / kKSt) & 1 : (vn / kVSt) & 1;
-            uint64_t* empty = pass == 0 ? &k_empty[st] : &v_empty[st];
-            uint64_t* full = pass == 0 ? &k_full[st] : &v_full[st];
-            uint8_t* dst = (pass == 0 ? sK : sV) + st * kKVBytes;
-            if (lane == 0) {
-              ok = mbar_wait(empty, ph ^ 1, &abort_flag);
-              if (ok) mbar_expect_tx(full, kKVBytes);
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (ok) {
-              // lane handles keys 4*lane .. 4*lane+3 of the tile
-              int rows[4];
-              bool win = false;
-              int fallback = -1;
+      const int b = it.kl.row / a.T;
+      for (int g0 = it.tile_beg; g0 < it.tile_end; g0 += kGT, ++G) {
+        const int nt = min(kGT, it.tile_end - g0);
+        const int slot = G % kTbl;
+        if (!mbar_wait(&t_empty[slot], empty_par(G, kTbl), &abort_flag)) break;
+        int src[kGT][4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                bool is_win;
-                const int src = key_source(a, it.kl, tile, 4 * lane + e, is_win, pass == 0);
-                win = is_win;
-                rows[e] = src;
-                if (src >= 0 && fallback < 0) fallback = src;
-              }
-              const int b = it.kl.row / a.T;
-              const int base = win ? b * a.ring : b * a.nc_cap;
-              if (fallback < 0) fallback = 0;
+        for (int j = 0; j < kGT; ++j)
 #pragma unroll
-              for (int e = 0; e < 4; ++e) rows[e] = base + (rows[e] >= 0 ? rows[e] : fallback);
-              const CUtensorMap* mp = pass == 0 ? (win ? &maps.kw : &maps.kc) : (win ? &maps.vw : &maps.vc);
+          for (int i = 0; i < 4; ++i) src[j][i] = j < nt ? key_source(a, it.kl, g0 + j, lane + 32 * i) : -1;
 #pragma unroll
-              for (int c = 0; c < 2; ++c)
-                tma_gather4(dst + c * (kKVBytes / 2) + lane * 4 * 128, mp, full, c * 64, rows[0], rows[1], rows[2],
-                            rows[3]);
-            }
-            if (pass == 0) ++kn; else ++vn;
+        for (int j = 0; j < kGT; ++j) {
+          if (j >= nt) break;
+          const bool win = g0 + j >= it.kl.comp_tiles;
+          const int base = win ? b * a.ring : b * a.nc_cap;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tbl.rows[slot][j * kTile + lane + 32 * i] = src[j][i] >= 0 ? base + src[j][i] : -1;
+          if (lane == 0) {
+            tbl.safe[slot][j] = base;
+            tbl.win[slot][j] = win ? 1 : 0;
           }
         }
+        mbar_arrive(&t_full[slot]);
+      }
+    }
+  } else if (warp == 0 || warp == 2) {
+    // ======================================================== K (+Q) and V producers
+    const bool is_k = warp == 0;
+    uint32_t G = 0, n = 0, tiles = 0;
+    bool ok = true;
+    if (lane == 0) {
+      prefetch_tmap(&maps.q); prefetch_tmap(&maps.kc); prefetch_tmap(&maps.kw);
+      prefetch_tmap(&maps.vc); prefetch_tmap(&maps.vw);
+    }
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      Item it;
+      it.init(a, w);
+      if (it.n_tiles() == 0) continue;
+      if (is_k) {
+        const int qb = n % kQSt;
+        if (lane == 0) {
+          ok = mbar_wait(&q_empty[qb], empty_par(n, kQSt), &abort_flag);
+          if (ok) {
+            mbar_expect_tx(&q_full[qb], kQBytes);
+            for (int c = 0; c < 2; ++c)
+              tma_load_2d(sQ + qb * kQBytes + c * (kQBytes / 2), &maps.q, &q_full[qb], c * 64, it.kl.row * kH);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+      ++n;
+      for (int g0 = it.tile_beg; g0 < it.tile_end && ok; g0 += kGT, ++G) {
+        const int nt = min(kGT, it.tile_end - g0);
+        const int slot = G % kTbl;
+        ok = mbar_wait(&t_full[slot], full_par(G, kTbl), &abort_flag);
+        for (int j = 0; j < nt && ok; ++j, ++tiles) {
+          const int st = tiles % 2;
+          uint64_t* empty = is_k ? &k_empty[st] : &v_empty[st];
+          uint64_t* full = is_k ? &k_full[st] : &v_full[st];
+          uint8_t* dst = (is_k ? sK : sV) + st * kKVBytes;
+          if (lane == 0) {
+            ok = mbar_wait(empty, empty_par(tiles, 2), &abort_flag);
+            if (ok) mbar_expect_tx(full, kKVBytes);
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          const int safe = tbl.safe[slot][j];
+          const bool win = tbl.win[slot][j] != 0;
+          int rows[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int rw = tbl.rows[slot][j * kTile + 4 * lane + e];
+            rows[e] = rw >= 0 ? rw : safe;
+          }
+          const CUtensorMap* mp = is_k ? (win ? &maps.kw : &maps.kc) : (win ? &maps.vw : &maps.vc);
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            tma_gather4(dst + c * (kKVBytes / 2) + lane * 4 * 128, mp, full, c * 64, rows[0], rows[1], rows[2], rows[3]);
+        }
+        mbar_arrive(&t_empty[slot]);
       }
     }
     // drain: loads in flight must land before the CTA can exit
     if (lane == 0 && abort_flag) {
       const unsigned long long t0 = globaltimer();
-      auto drain = [&](uint64_t* bars, int nst, uint32_t n) {
-        for (int s = 0; s < nst && (uint32_t)s < n; ++s) {
-          const uint32_t last = s + nst * ((n - 1 - s) / nst);
-          while (!mbar_try_wait(&bars[s], (last / nst) & 1) && globaltimer() - t0 < kWaitNs) {}
+      uint64_t* fulls = is_k ? k_full : v_full;
+      for (uint32_t s = 0; s < 2 && s < tiles; ++s) {
+        const uint32_t last = s + 2 * ((tiles - 1 - s) / 2);
+        while (!mbar_try_wait(&fulls[s], full_par(last, 2)) && globaltimer() - t0 < kWaitNs) {}
+      }
+      if (is_k)
+        for (uint32_t s = 0; s < kQSt && s < n; ++s) {
+          const uint32_t last = s + kQSt * ((n - 1 - s) / kQSt);
+          while (!mbar_try_wait(&q_full[s], full_par(last, kQSt)) && globaltimer() - t0 < kWaitNs) {}
         }
-      };
-      drain(k_full, kKSt, kn);
-      drain(v_full, kVSt, vn);
-      if (qn > 0) while (!mbar_try_wait(&q_full, (qn - 1) & 1) && globaltimer() - t0 < kWaitNs) {}
     }
   } else if (warp == 1) {
     // ======================================================== MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc1 = idesc_bf16_f32(128, kH, false, false);
       constexpr uint32_t idesc2 = idesc_bf16_f32(128, kH, true, true);
-      uint32_t qn = 0, kn = 0, vn = 0, pn = 0, gn = 0, on = 0;
+      uint32_t G = 0, n = 0, kt = 0, vt = 0, pt = 0;
+      uint32_t ordy[2] = {0, 0};
+      PendingPV pend{0, 0, 0, 0};
       bool ok = true;
+      auto issue_pv = [&](const PendingPV& pv) {
+        if (!ok) return;
+        ok = mbar_wait(&o_ready[pv.ob], full_par(ordy[pv.ob], 1), &abort_flag);
+        ++ordy[pv.ob];
+        for (int j = 0; j < pv.ntiles && ok; ++j) {
+          const int vs = vt % kVSt, ps = pt % kPSt;
+          ok = mbar_wait(&v_full[vs], full_par(vt, kVSt), &abort_flag) &&
+               mbar_wait(&p_full[ps], full_par(pt, kPSt), &abort_flag);
+          if (!ok) break;
+          fence_after_sync();
+          const uint32_t vbase = smem_u32(sV + vs * kKVBytes);
+          const uint32_t pbase = smem_u32(sP + ps * kPBytes);
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_f16_ss(tmem + kOCol + pv.ob * kH, desc_mnmajor_sw128(vbase + kk * 2048, kKVBytes / 2),
+                       desc_mnmajor_sw128(pbase + kk * 2048, 0), idesc2, (pv.first && j == 0 && kk == 0) ? 0u : 1u);
+          mma_commit(&v_empty[vs]);
+          mma_commit(&p_empty[ps]);
+          ++vt;
+          ++pt;
+        }
+        mma_commit(&o_full[pv.ob]);
+      };
       for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
         Item it;
         it.init(a, w);
         if (it.n_tiles() == 0) continue;
-        ok = mbar_wait(&q_full, qn & 1, &abort_flag);
-        ++qn;
-        bool first_pv = true;
-        for (int g0 = it.tile_beg; g0 < it.tile_end && ok; g0 += kGroup) {
-          const int g1 = min(it.tile_end, g0 + kGroup);
-          // S^T tiles of the group (after the softmax released the previous group's)
-          ok = mbar_wait(&s_free, (gn & 1) ^ 1, &abort_flag);
-          for (int tile = g0; tile < g1 && ok; ++tile) {
-            const int st = kn % kKSt;
-            ok = mbar_wait(&k_full[st], (kn / kKSt) & 1, &abort_flag);
+        const int qb = n % kQSt, ob = n % 2;
+        bool first = true;
+        for (int g0 = it.tile_beg; g0 < it.tile_end && ok; g0 += kGT, ++G) {
+          const int nt = min(kGT, it.tile_end - g0);
+          const bool last = g0 + kGT >= it.tile_end;
+          const int sb = G % 2;
+          ok = mbar_wait(&s_free[sb], empty_par(G, 2), &abort_flag);
+          if (ok && first) ok = mbar_wait(&q_full[qb], full_par(n, kQSt), &abort_flag);
+          for (int j = 0; j < nt && ok; ++j, ++kt) {
+            const int ks = kt % kKSt;
+            ok = mbar_wait(&k_full[ks], full_par(kt, kKSt), &abort_flag);
             if (!ok) break;
             fence_after_sync();
-            const uint32_t d = tmem + (tile - g0) * kH;
-            const uint32_t kbase = smem_u32(sK + st * kKVBytes);
-            const uint32_t qbase = smem_u32(sQ);
+            const uint32_t d = tmem + sb * kSCols + j * kH;
+            const uint32_t kbase = smem_u32(sK + ks * kKVBytes);
+            const uint32_t qbase = smem_u32(sQ + qb * kQBytes);
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 mma_f16_ss(d, desc_kmajor_sw128(kbase + c * (kKVBytes / 2) + kk * 32),
                            desc_kmajor_sw128(qbase + c * (kQBytes / 2) + kk * 32), idesc1, (c | kk) != 0);
-            mma_commit(&k_empty[st]);
-            ++kn;
+            mma_commit(&k_empty[ks]);
           }
-          for (int j = 0; j < kGroup; ++j) mma_commit(&s_full[j]);
-          if (g1 == it.tile_end) mma_commit(&q_empty);
-          ++gn;
-          // O^T += V^T P^T over the group's tiles
-          if (ok) ok = mbar_wait(&o_ready, on & 1, &abort_flag);
-          ++on;
-          for (int tile = g0; tile < g1 && ok; ++tile) {
-            const int vs = vn % kVSt, ps = pn % kPSt;
-            ok = mbar_wait(&v_full[vs], (vn / kVSt) & 1, &abort_flag) &&
-                 mbar_wait(&p_full[ps], (pn / kPSt) & 1, &abort_flag);
-            if (!ok) break;
-            fence_after_sync();
-            const uint32_t vbase = smem_u32(sV + vs * kKVBytes);
-            const uint32_t pbase = smem_u32(sP + ps * kPBytes);
-#pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk) {
-              mma_f16_ss(tmem + kOCol, desc_mnmajor_sw128(vbase + kk * 2048, kKVBytes / 2),
-                         desc_mnmajor_sw128(pbase + kk * 2048, 0), idesc2, (first_pv && kk == 0) ? 0u : 1u);
-            }
-            first_pv = false;
-            mma_commit(&v_empty[vs]);
-            mma_commit(&p_empty[ps]);
-            ++vn;
-            ++pn;
-          }
-          mma_commit(&o_full);
+          mma_commit(&s_full[sb]);
+          if (last) mma_commit(&q_empty[qb]);
+          if (pend.valid) issue_pv(pend);
+          pend = PendingPV{1, ob, nt, first ? 1 : 0};
+          first = false;
         }
+        ++n;
       }
+      if (pend.valid) issue_pv(pend);
       mma_commit(&mma_done);
       const unsigned long long t0 = globaltimer();
       while (!mbar_try_wait(&mma_done, 0) && globaltimer() - t0 < kWaitNs) {}
     }
+  }
   } else {
-    // ======================================================== softmax + epilogue
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+    // ======================================================== softmax + epilogue (warps 4..11)
     const int quad = warp & 3;
-    const int kk = quad * 32 + lane;                  // key lane within a tile / d for O^T
+    const int hf = (warp - 4) >> 2;                   // head half: heads 32*hf .. 32*hf+31
+    const int kk = quad * 32 + lane;                  // key lane of a tile; head-dim lane of O^T
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const int st = tid - 64;                          // 0..127 among the softmax threads
-    uint32_t gn = 0, pn = 0, on = 0;
+    uint32_t G = 0, n = 0, pt = 0;
+    uint32_t ofw[2] = {0, 0};
     bool ok = true;   // on a failed wait the warps keep the same control flow (named barriers) and skip work
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
       Item it;
       it.init(a, w);
+      const bool final_out = a.nsplit == 1;
+      const size_t prow = final_out ? (size_t)it.kl.row * kH : ((size_t)it.kl.row * a.nsplit + it.split) * kH;
       if (it.n_tiles() == 0) {
-        // nothing visible at all (cannot happen with W >= 1): write an empty result
-        if (a.nsplit == 1) {
-          for (int h = 0; h < kH; ++h) store_f((bf16*)a.o + ((size_t)it.kl.row * kH + h) * kD + kk, 0.f);
-          if (a.lse && st < kH) a.lse[(size_t)it.kl.row * kH + st] = -INFINITY;
-        } else {
-          const size_t prow = ((size_t)it.kl.row * a.nsplit + it.split) * kH;
-          for (int h = 0; h < kH; ++h) a.part_o[(prow + h) * kD + kk] = 0.f;
-          if (st < kH) a.part_lse[prow + st] = -INFINITY;
+        // no key at all (impossible with W >= 1 in prefill; empty slices in split-KV)
+#pragma unroll 4
+        for (int e = 0; e < 32; ++e) {
+          const int h = hf * 32 + e;
+          if (final_out) store_f((bf16*)a.o + (prow + h) * kD + kk, 0.f);
+          else a.part_o[(prow + h) * kD + kk] = 0.f;
+        }
+        if (quad == 0) {
+          const int h = hf * 32 + lane;
+          if (final_out) { if (a.lse) a.lse[prow + h] = -INFINITY; }
+          else a.part_lse[prow + h] = -INFINITY;
         }
         continue;
       }
-      if (st < kH) m_run[st] = -INFINITY;
-      float lp[kH];
+      const int ob = n % 2;
+      float lp[32];
 #pragma unroll
-      for (int h = 0; h < kH; ++h) lp[h] = 0.f;
-      bool first_group = true;
-      for (int g0 = it.tile_beg; g0 < it.tile_end; g0 += kGroup) {
-        const int g1 = min(it.tile_end, g0 + kGroup);
-        // ---- pass A: elementwise max over the group's tiles
-        float mx[kH];
+      for (int e = 0; e < 32; ++e) lp[e] = 0.f;
+      bool first = true;
+      for (int g0 = it.tile_beg; g0 < it.tile_end; g0 += kGT, ++G) {
+        const int nt = min(kGT, it.tile_end - g0);
+        const bool last = g0 + kGT >= it.tile_end;
+        const int sb = G % 2, slot = G % kTbl;
+        ok = mbar_wait(&t_full[slot], full_par(G, kTbl), &abort_flag) && ok;
+        uint32_t vmask = 0;   // bit j: this thread's key of tile j is a real key
 #pragma unroll
-        for (int h = 0; h < kH; ++h) mx[h] = -INFINITY;
-        for (int tile = g0; tile < g1; ++tile) {
-          ok = mbar_wait(&s_full[tile - g0], gn & 1, &abort_flag) && ok;
+        for (int j = 0; j < kGT; ++j) vmask |= (j < nt && tbl.rows[slot][j * kTile + kk] >= 0) ? (1u << j) : 0u;
+        mbar_arrive(&t_empty[slot]);
+        ok = mbar_wait(&s_full[sb], full_par(G, 2), &abort_flag) && ok;
+        fence_after_sync();
+        // ---- pass A: elementwise max over the group's tiles, then across key lanes
+        float mx[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx[e] = -INFINITY;
+#pragma unroll 1
+        for (int j = 0; j < nt; ++j) {
+          uint32_t v[32];
+          tmem_ld32(lane_addr + sb * kSCols + j * kH + hf * 32, v);
+          tmem_wait_ld();
+          if (vmask & (1u << j)) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) mx[e] = fmaxf(mx[e], __uint_as_float(v[e]));
+          }
+        }
+        warp_xmax32(mx, lane);
+        red[hf][quad][lane] = mx[0] * c2;
+        named_sync_softmax();
+        if (quad == 0) {
+          const int h = hf * 32 + lane;
+          const float g = fmaxf(fmaxf(red[hf][0][lane], red[hf][1][lane]), fmaxf(red[hf][2][lane], red[hf][3][lane]));
+          const float mo = m_run[h];
+          float mn = mo, al = 1.f;
+          bool resc = false;
+          if (first) {
+            mn = g;
+          } else if (g > mo + kRescaleThreshold || (mo == -INFINITY && g != -INFINITY)) {
+            mn = g;
+            al = mo == -INFINITY ? 0.f : ex2_approx(mo - mn);
+            resc = true;
+          }
+          m_run[h] = mn;
+          m_use[h] = mn == -INFINITY ? 0.f : mn;
+          alpha_s[h] = al;
+          const unsigned any = __ballot_sync(0xffffffffu, resc);
+          if (lane == 0) resc_flag[hf] = any != 0;
+        }
+        named_sync_softmax();
+        // ---- O^T of the previous group of this query is complete; rescale if needed
+        if (!first) {
+          ok = mbar_wait(&o_full[ob], full_par(ofw[ob], 1), &abort_flag) && ok;
+          ++ofw[ob];
           fence_after_sync();
-          bool is_win;
-          const bool valid = key_source(a, it.kl, tile, kk, is_win, false) >= 0;
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
+          if (resc_flag[hf]) {
             uint32_t v[32];
-            tmem_ld32(lane_addr + (tile - g0) * kH + c * 32, v);
+            const uint32_t oaddr = lane_addr + kOCol + ob * kH + hf * 32;
+            tmem_ld32(oaddr, v);
             tmem_wait_ld();
-            if (valid) {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) mx[c * 32 + e] = fmaxf(mx[c * 32 + e], __uint_as_float(v[e]));
+            for (int e = 0; e < 32; ++e) {
+              const float al = alpha_s[hf * 32 + e];
+              v[e] = __float_as_uint(__uint_as_float(v[e]) * al);
+              lp[e] *= al;
             }
+            tmem_st32(oaddr, v);
+            tmem_wait_st();
           }
-        }
-        warp_xmax64(mx, lane);
-        red[quad][2 * lane] = mx[0];
-        red[quad][2 * lane + 1] = mx[1];
-        named_sync_softmax();
-        if (st < kH) {
-          const float mg = fmaxf(fmaxf(red[0][st], red[1][st]), fmaxf(red[2][st], red[3][st]));
-          const float mo = m_run[st];
-          const float mn = fmaxf(mo, mg);
-          alpha[st] = (mn == -INFINITY || mo == -INFINITY) ? (mo == -INFINITY ? 0.f : 1.f) : exp2f((mo - mn) * c2);
-          m_run[st] = mn;
-          m_use[st] = mn == -INFINITY ? 0.f : mn * c2;   // pre-multiplied by scale*log2(e)
-        }
-        named_sync_softmax();
-        // ---- rescale the running O^T and partial sums when a later group raised the max
-        if (!first_group) {
-          ok = mbar_wait(&o_full, (on & 1), &abort_flag) && ok;  // previous group's PV finished
-          ++on;
-          fence_after_sync();
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t v[32];
-            tmem_ld32(lane_addr + kOCol + c * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha[c * 32 + e]);
-            tmem_st32(lane_addr + kOCol + c * 32, v);
-          }
-          tmem_wait_st();
-#pragma unroll
-          for (int h = 0; h < kH; ++h) lp[h] *= alpha[h];
         }
         fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&o_ready);
-        // ---- pass B: probabilities
-        for (int tile = g0; tile < g1; ++tile) {
-          bool is_win;
-          const bool valid = key_source(a, it.kl, tile, kk, is_win, false) >= 0;
-          const int ps = pn % kPSt;
-          ok = mbar_wait(&p_empty[ps], ((pn / kPSt) & 1) ^ 1, &abort_flag) && ok;
-          uint8_t* prow = sP + ps * kPBytes + kk * 128;
+        if (lane == 0) mbar_arrive(&o_ready[ob]);
+        // ---- pass B: probabilities into P^T
+        const float* mu = m_use + hf * 32;
+#pragma unroll 1
+        for (int j = 0; j < nt; ++j) {
+          const int ps = pt % kPSt;
+          ok = mbar_wait(&p_empty[ps], empty_par(pt, kPSt), &abort_flag) && ok;
+          uint32_t v[32];
+          tmem_ld32(lane_addr + sb * kSCols + j * kH + hf * 32, v);
+          tmem_wait_ld();
+          uint32_t pk[16];
+          const bool valid = (vmask >> j) & 1u;
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t v[32];
-            tmem_ld32(lane_addr + (tile - g0) * kH + c * 32, v);
-            tmem_wait_ld();
-            uint32_t pk[16];
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = valid ? ex2_approx(fmaf(__uint_as_float(v[e]), c2, -mu[e])) : 0.f;
+            const float p1 = valid ? ex2_approx(fmaf(__uint_as_float(v[e + 1]), c2, -mu[e + 1])) : 0.f;
+            lp[e] += p0;
+            lp[e + 1] += p1;
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+            pk[e / 2] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          uint8_t* prow_s = sP + ps * kPBytes + kk * 128;
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float p0 = valid ? exp2f(fmaf(__uint_as_float(v[e]), c2, -m_use[c * 32 + e])) : 0.f;
-              const float p1 = valid ? exp2f(fmaf(__uint_as_float(v[e + 1]), c2, -m_use[c * 32 + e + 1])) : 0.f;
-              lp[c * 32 + e] += p0;
-              lp[c * 32 + e + 1] += p1;
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-              pk[e / 2] = *reinterpret_cast<uint32_t*>(&b2);
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {  // 16-byte chunks (8 heads) 4c+q of this key's row
-              const int chunk = (c * 4 + q) ^ (kk & 7);
-              *reinterpret_cast<uint4*>(prow + chunk * 16) =
-                  make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-            }
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = (hf * 4 + q) ^ (kk & 7);
+            *reinterpret_cast<uint4*>(prow_s + chunk * 16) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_full[ps]);
-          ++pn;
+          ++pt;
         }
         fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free);
-        ++gn;
-        first_group = false;
-      }
-      // ---- epilogue: l = sum over lanes of lp; o = O^T / l
-      warp_xsum64(lp, lane);
-      red[quad][2 * lane] = lp[0];
-      red[quad][2 * lane + 1] = lp[1];
-      named_sync_softmax();
-      if (st < kH) l_fin[st] = red[0][st] + red[1][st] + red[2][st] + red[3][st];
-      named_sync_softmax();
-      ok = mbar_wait(&o_full, on & 1, &abort_flag) && ok;
-      ++on;
-      fence_after_sync();
-      const bool final_out = a.nsplit == 1;
-      const size_t prow = ((size_t)it.kl.row * a.nsplit + it.split) * kH;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
+        if (lane == 0) mbar_arrive(&s_free[sb]);
+        first = false;
+        if (!last) continue;
+        // ---- epilogue of the item: l = sum over key lanes; o = O^T / l
+        ok = mbar_wait(&o_full[ob], full_par(ofw[ob], 1), &abort_flag) && ok;
+        ++ofw[ob];
+        fence_after_sync();
+        warp_xsum32(lp, lane);
+        red[hf][quad][lane] = lp[0];
+        named_sync_softmax();
+        if (quad == 0) {
+          const int h = hf * 32 + lane;
+          const float l = red[hf][0][lane] + red[hf][1][lane] + red[hf][2][lane] + red[hf][3][lane];
+          l_fin[h] = l;
+          const float lse = l > 0.f ? m_run[h] * 0.6931471805599453f + logf(l) : -INFINITY;
+          if (final_out) { if (a.lse) a.lse[prow + h] = lse; }
+          else a.part_lse[prow + h] = lse;
+        }
+        named_sync_softmax();
         uint32_t v[32];
-        tmem_ld32(lane_addr + kOCol + c * 32, v);
+        tmem_ld32(lane_addr + kOCol + ob * kH + hf * 32, v);
         tmem_wait_ld();
-#pragma unroll
+#pragma unroll 4
         for (int e = 0; e < 32; ++e) {
-          const int h = c * 32 + e;
+          const int h = hf * 32 + e;
           const float l = l_fin[h];
           const float o = l > 0.f ? __uint_as_float(v[e]) / l : 0.f;
-          if (final_out) store_f((bf16*)a.o + ((size_t)it.kl.row * kH + h) * kD + kk, o);
+          if (final_out) store_f((bf16*)a.o + (prow + h) * kD + kk, o);
           else a.part_o[(prow + h) * kD + kk] = o;
         }
+        fence_before_sync();
+        named_sync_softmax();   // l_fin / m_run are rewritten by the next item
       }
-      if (st < kH) {
-        const float l = l_fin[st];
-        const float lse = l > 0.f ? m_run[st] * a.scale + logf(l) : -INFINITY;
-        if (final_out) { if (a.lse) a.lse[(size_t)it.kl.row * kH + st] = lse; }
-        else a.part_lse[prow + st] = lse;
-      }
-      fence_before_sync();
-      named_sync_softmax();   // everyone done with m_run / l_fin / O^T before the next item
+      ++n;
     }
   }
   fence_before_sync();
@@ -508,8 +594,8 @@ inline cudaError_t launch_attn_tc(const AttnArgs& a, int batch, cudaStream_t str
   using namespace attn_tc;
   Maps m;
   const uint64_t rows_q = (uint64_t)batch * a.T * kH;
-  // Padding keys gather row 0 of their source; with no compressed cache at all the
-  // compressed maps point at the window ring so that row stays inside an allocation.
+  // Masked keys gather a row of their own source; with no compressed cache at all
+  // the compressed maps point at the window ring so that row stays in an allocation.
   const bool no_cache = a.kc == nullptr || a.vc == nullptr || a.nc_cap <= 0;
   const void* kc = no_cache ? a.kw : a.kc;
   const void* vc = no_cache ? a.vw : a.vc;
@@ -519,6 +605,8 @@ inline cudaError_t launch_attn_tc(const AttnArgs& a, int batch, cudaStream_t str
   if (!make_map_bf16_2d(&m.vc, vc, rows_c, kD, kD * 2, 1, 64)) return cudaErrorInvalidValue;
   if (!make_map_bf16_2d(&m.kw, a.kw, (uint64_t)batch * a.ring, kD, kD * 2, 1, 64)) return cudaErrorInvalidValue;
   if (!make_map_bf16_2d(&m.vw, a.vw, (uint64_t)batch * a.ring, kD, kD * 2, 1, 64)) return cudaErrorInvalidValue;
+  AttnArgs aa = a;
+  if (no_cache) aa.nc_cap = 0;   // compressed rows then index the ring map from row b*0
   const int n_items = batch * a.T * a.nsplit;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -526,7 +614,7 @@ inline cudaError_t launch_attn_tc(const AttnArgs& a, int batch, cudaStream_t str
   const int grid = n_items < sms ? n_items : sms;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<<<grid, kThreads, kSmem, stream>>>(m, a, n_items);
+  attn_tc_kernel<<<grid, kThreads, kSmem, stream>>>(m, aa, n_items);
   count_launch();
   return cudaGetLastError();
 }
