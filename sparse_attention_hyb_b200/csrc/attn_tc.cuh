@@ -9,19 +9,24 @@
 // A query's keys (compressed entries first, then window positions, each padded
 // to whole tiles of 128) are processed in groups of up to 3 tiles.
 //
-// Roles (12 warps, one CTA per SM, persistent over work items):
-//   warp 3      key tables: turns each group's key list (indexer output or the
+// Roles (16 warps, one CTA per SM, persistent over work items):
+//   warp 1      key tables: turns each group's key list (indexer output or the
 //               dense range, then the window) into source rows in shared memory
-//               one group ahead, so no role waits on a global index load;
-//   warp 0      Q (2-D TMA, double-buffered) and K tiles (TMA gather4, 4 rows
-//               per instruction, every lane issuing its own rows);
-//   warp 2      V tiles (TMA gather4);
-//   warp 1      TMEM owner; one thread issues every MMA: S^T of group g+1 is
+//               one group ahead, so no role waits on a global index load; also
+//               loads each query's Q tile (2-D TMA, double-buffered);
+//   warps 2-4   K tiles, warps 5-7 V tiles: gathered rows are copied with
+//               16-byte cp.async by all 96 lanes (the per-SM gather rate grows
+//               with the number of issuing warps), written in the 128-byte
+//               swizzled layout; a window tile whose rows are consecutive is one
+//               2-D TMA box per 64-column half instead.  Every producer lane
+//               makes one asynchronous arrival per tile that the hardware
+//               performs when the lane's copies have landed;
+//   warp 0      TMEM owner; one thread issues every MMA: S^T of group g+1 is
 //               issued before O^T of group g, so the tensor core computes the
 //               next group's scores while the softmax warps turn the current
 //               scores into probabilities;
-//   warps 4..11 softmax and epilogue: thread = key lane (TMEM lane quadrant =
-//               warp % 4), warps 4-7 own heads 0-31 and warps 8-11 heads 32-63.
+//   warps 8-15  softmax and epilogue: thread = key lane (TMEM lane quadrant =
+//               warp % 4), warps 8-11 own heads 0-31 and warps 12-15 heads 32-63.
 // Tensor memory: two S^T buffers (3 tiles x 64 columns) and two O^T
 // accumulators (64 columns), 512 columns in all.
 //
@@ -46,7 +51,9 @@ namespace attn_tc {
 constexpr int kH = 64, kD = 128, kTile = 128;
 constexpr int kGT = 3;                                  // tiles per group
 constexpr int kQSt = 2, kKSt = 2, kVSt = 2, kPSt = 2, kTbl = 4;
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+constexpr int kProdWarps = 3;                           // per tensor (K, V)
+constexpr int kProdLanes = kProdWarps * 32;
 constexpr int kQBytes = kH * kD * 2;                    // 16 KB, two 64-column sub-tiles
 constexpr int kKVBytes = kTile * kD * 2;                // 32 KB, two 64-column sub-tiles
 constexpr int kPBytes = kTile * kH * 2;                 // 16 KB
@@ -54,10 +61,11 @@ constexpr int kSmem = kQSt * kQBytes + kKSt * kKVBytes + kVSt * kKVBytes + kPSt 
 constexpr uint32_t kSCols = kGT * kH;                   // 192 columns per S^T buffer
 constexpr uint32_t kOCol = 2 * kSCols;                  // O^T buffers at 384 and 448
 constexpr float kRescaleThreshold = 8.f;                // base-2 units
-constexpr int kTblArrivals = 32 + 32 + 256;             // K producer, V producer, softmax lanes
+constexpr int kTblArrivals = 2 * kProdLanes + 256;      // K producers, V producers, softmax lanes
 
 struct Maps {
-  CUtensorMap q, kc, vc, kw, vw;
+  CUtensorMap q;        // [batch*T*H, D], 64 x 64 boxes
+  CUtensorMap kw, vw;   // [batch*ring, D], 128-row x 64-column boxes (contiguous window tiles)
 };
 
 // Per-query key list: compressed slots [0, n_comp) padded to whole tiles, then
@@ -112,9 +120,10 @@ __device__ __forceinline__ int key_source(const AttnArgs& a, const KeyList& kl, 
 }
 
 struct KeyTable {
-  int rows[kTbl][kGT * kTile];   // source row in the gather map, -1 = masked key
-  int safe[kTbl][kGT];           // a row inside the map for masked keys of the tile
+  int rows[kTbl][kGT * kTile];   // source row, -1 = masked key
+  int safe[kTbl][kGT];           // a real row of the tile's source for masked keys
   int win[kTbl][kGT];            // 1 if the tile holds window keys
+  int first[kTbl][kGT];          // >= 0: the tile is rows first .. first+127 of the window source
 };
 
 __device__ __forceinline__ void named_sync_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -202,8 +211,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   if (tid == 0) {
     abort_flag = 0;
     for (int s = 0; s < kQSt; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
-    for (int s = 0; s < kKSt; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
-    for (int s = 0; s < kVSt; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
+    for (int s = 0; s < kKSt; ++s) { mbar_init(&k_full[s], kProdLanes); mbar_init(&k_empty[s], 1); }
+    for (int s = 0; s < kVSt; ++s) { mbar_init(&v_full[s], kProdLanes); mbar_init(&v_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1); mbar_init(&s_free[s], 8);
       mbar_init(&o_full[s], 1); mbar_init(&o_ready[s], 8);
@@ -213,24 +222,32 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     mbar_init(&mma_done, 1);
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(&tmem_base, 512);
+  if (warp == 0) tmem_alloc(&tmem_base, 512);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = tmem_base;
   const float c2 = a.scale * 1.4426950408889634f;  // scale * log2(e)
 
-  // Register split per warpgroup.  Launch: 384 threads x 168 = 64512 registers;
-  // after the split 128 x 88 + 256 x 200 = 62464, within the launch's total.
-  if (warp < 4) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
-  if (warp == 3) {
-    // ======================================================== key tables
-    uint32_t G = 0;
+  // Register split per warpgroup.  Launch: 512 threads x 128 = 65536 registers;
+  // after the split 256 x 56 (warps 0-7) + 256 x 200 (warps 8-15) = 65536.
+  if (warp < 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+  if (warp == 1) {
+    // ======================================================== key tables and Q
+    uint32_t G = 0, n = 0;
     for (int w = blockIdx.x; w < n_items && !abort_flag; w += gridDim.x) {
       Item it;
       it.init(a, w);
+      if (it.n_tiles() == 0) continue;
       const int b = it.kl.row / a.T;
+      const int qb = n % kQSt;
+      if (lane == 0 && mbar_wait(&q_empty[qb], empty_par(n, kQSt), &abort_flag)) {
+        mbar_expect_tx(&q_full[qb], kQBytes);
+        for (int c = 0; c < 2; ++c)
+          tma_load_2d(sQ + qb * kQBytes + c * (kQBytes / 2), &maps.q, &q_full[qb], c * 64, it.kl.row * kH);
+      }
+      ++n;
       for (int g0 = it.tile_beg; g0 < it.tile_end; g0 += kGT, ++G) {
         const int nt = min(kGT, it.tile_end - g0);
         const int slot = G % kTbl;
@@ -250,37 +267,28 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           if (lane == 0) {
             tbl.safe[slot][j] = base;
             tbl.win[slot][j] = win ? 1 : 0;
+            int first = -1;
+            if (win) {   // window positions are consecutive rows unless the ring wraps inside the tile
+              const int s0 = (it.kl.w0 + (g0 + j - it.kl.comp_tiles) * kTile) % a.ring;
+              if (s0 + kTile <= a.ring) first = base + s0;
+            }
+            tbl.first[slot][j] = first;
           }
         }
         mbar_arrive(&t_full[slot]);
       }
     }
-  } else if (warp == 0 || warp == 2) {
-    // ======================================================== K (+Q) and V producers
-    const bool is_k = warp == 0;
-    uint32_t G = 0, n = 0, tiles = 0;
+  } else if (warp >= 2) {
+    // ======================================================== K (warps 2-4) and V (warps 5-7) producers
+    const bool is_k = warp < 2 + kProdWarps;
+    const int plane = (warp - (is_k ? 2 : 2 + kProdWarps)) * 32 + lane;   // 0 .. kProdLanes-1
+    uint32_t G = 0, tiles = 0;
     bool ok = true;
-    if (lane == 0) {
-      prefetch_tmap(&maps.q); prefetch_tmap(&maps.kc); prefetch_tmap(&maps.kw);
-      prefetch_tmap(&maps.vc); prefetch_tmap(&maps.vw);
-    }
+    if (plane == 0) prefetch_tmap(is_k ? &maps.kw : &maps.vw);
     for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
       Item it;
       it.init(a, w);
       if (it.n_tiles() == 0) continue;
-      if (is_k) {
-        const int qb = n % kQSt;
-        if (lane == 0) {
-          ok = mbar_wait(&q_empty[qb], empty_par(n, kQSt), &abort_flag);
-          if (ok) {
-            mbar_expect_tx(&q_full[qb], kQBytes);
-            for (int c = 0; c < 2; ++c)
-              tma_load_2d(sQ + qb * kQBytes + c * (kQBytes / 2), &maps.q, &q_full[qb], c * 64, it.kl.row * kH);
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-      }
-      ++n;
       for (int g0 = it.tile_beg; g0 < it.tile_end && ok; g0 += kGT, ++G) {
         const int nt = min(kGT, it.tile_end - g0);
         const int slot = G % kTbl;
@@ -290,43 +298,44 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           uint64_t* empty = is_k ? &k_empty[st] : &v_empty[st];
           uint64_t* full = is_k ? &k_full[st] : &v_full[st];
           uint8_t* dst = (is_k ? sK : sV) + st * kKVBytes;
-          if (lane == 0) {
-            ok = mbar_wait(empty, empty_par(tiles, 2), &abort_flag);
-            if (ok) mbar_expect_tx(full, kKVBytes);
-          }
+          if (lane == 0) ok = mbar_wait(empty, empty_par(tiles, 2), &abort_flag);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
-          const int safe = tbl.safe[slot][j];
-          const bool win = tbl.win[slot][j] != 0;
-          int rows[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int rw = tbl.rows[slot][j * kTile + 4 * lane + e];
-            rows[e] = rw >= 0 ? rw : safe;
+          const int first = tbl.first[slot][j];
+          if (first >= 0) {
+            // consecutive window rows: one 2-D TMA box per 64-column half
+            if (plane == 0) {
+              mbar_expect_tx_only(full, kKVBytes);
+              for (int c = 0; c < 2; ++c)
+                tma_load_2d(dst + c * (kKVBytes / 2), is_k ? &maps.kw : &maps.vw, full, c * 64, first);
+            }
+          } else {
+            // gathered rows: 16-byte cp.async per lane, lane-consecutive chunks of a
+            // 256-byte row, written with the 128-byte swizzle the MMA descriptors expect
+            const int safe = tbl.safe[slot][j];
+            const bool win = tbl.win[slot][j] != 0;
+            const char* src = static_cast<const char*>(is_k ? (win ? a.kw : a.kc) : (win ? a.vw : a.vc));
+            const int* trow = tbl.rows[slot] + j * kTile;
+            const uint32_t dbase = smem_u32(dst);
+#pragma unroll 4
+            for (int i = 0; i < (kTile * 16 + kProdLanes - 1) / kProdLanes; ++i) {
+              const int q = i * kProdLanes + plane;
+              if (q < kTile * 16) {
+                const int r = q >> 4, c = (q >> 3) & 1, ch = q & 7;
+                int rw = trow[r];
+                rw = rw >= 0 ? rw : safe;
+                cp_async16(dbase + c * (kKVBytes / 2) + r * 128 + ((ch ^ (r & 7)) << 4),
+                           src + (size_t)rw * (kD * 2) + c * 128 + ch * 16);
+              }
+            }
           }
-          const CUtensorMap* mp = is_k ? (win ? &maps.kw : &maps.kc) : (win ? &maps.vw : &maps.vc);
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            tma_gather4(dst + c * (kKVBytes / 2) + lane * 4 * 128, mp, full, c * 64, rows[0], rows[1], rows[2], rows[3]);
+          cp_async_arrive_noinc(full);   // arrives when this lane's copies of the tile have landed
         }
         mbar_arrive(&t_empty[slot]);
       }
     }
-    // drain: loads in flight must land before the CTA can exit
-    if (lane == 0 && abort_flag) {
-      const unsigned long long t0 = globaltimer();
-      uint64_t* fulls = is_k ? k_full : v_full;
-      for (uint32_t s = 0; s < 2 && s < tiles; ++s) {
-        const uint32_t last = s + 2 * ((tiles - 1 - s) / 2);
-        while (!mbar_try_wait(&fulls[s], full_par(last, 2)) && globaltimer() - t0 < kWaitNs) {}
-      }
-      if (is_k)
-        for (uint32_t s = 0; s < kQSt && s < n; ++s) {
-          const uint32_t last = s + kQSt * ((n - 1 - s) / kQSt);
-          while (!mbar_try_wait(&q_full[s], full_par(last, kQSt)) && globaltimer() - t0 < kWaitNs) {}
-        }
-    }
-  } else if (warp == 1) {
+    cp_async_wait<0>();
+  } else {
     // ======================================================== MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc1 = idesc_bf16_f32(128, kH, false, false);
@@ -345,6 +354,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
                mbar_wait(&p_full[ps], full_par(pt, kPSt), &abort_flag);
           if (!ok) break;
           fence_after_sync();
+          fence_async_shared();
           const uint32_t vbase = smem_u32(sV + vs * kKVBytes);
           const uint32_t pbase = smem_u32(sP + ps * kPBytes);
 #pragma unroll
@@ -375,6 +385,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
             ok = mbar_wait(&k_full[ks], full_par(kt, kKSt), &abort_flag);
             if (!ok) break;
             fence_after_sync();
+            fence_async_shared();
             const uint32_t d = tmem + sb * kSCols + j * kH;
             const uint32_t kbase = smem_u32(sK + ks * kKVBytes);
             const uint32_t qbase = smem_u32(sQ + qb * kQBytes);
@@ -402,9 +413,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
-    // ======================================================== softmax + epilogue (warps 4..11)
+    // ======================================================== softmax + epilogue (warps 8..15)
     const int quad = warp & 3;
-    const int hf = (warp - 4) >> 2;                   // head half: heads 32*hf .. 32*hf+31
+    const int hf = (warp - 8) >> 2;                   // head half: heads 32*hf .. 32*hf+31
     const int kk = quad * 32 + lane;                  // key lane of a tile; head-dim lane of O^T
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     uint32_t G = 0, n = 0, pt = 0;
@@ -578,7 +589,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace attn_tc
@@ -594,19 +605,17 @@ inline cudaError_t launch_attn_tc(const AttnArgs& a, int batch, cudaStream_t str
   using namespace attn_tc;
   Maps m;
   const uint64_t rows_q = (uint64_t)batch * a.T * kH;
-  // Masked keys gather a row of their own source; with no compressed cache at all
-  // the compressed maps point at the window ring so that row stays in an allocation.
-  const bool no_cache = a.kc == nullptr || a.vc == nullptr || a.nc_cap <= 0;
-  const void* kc = no_cache ? a.kw : a.kc;
-  const void* vc = no_cache ? a.vw : a.vc;
-  const uint64_t rows_c = no_cache ? (uint64_t)batch * a.ring : (uint64_t)batch * a.nc_cap;
   if (!make_map_bf16_2d(&m.q, a.q, rows_q, kD, kD * 2, 64, 64)) return cudaErrorInvalidValue;
-  if (!make_map_bf16_2d(&m.kc, kc, rows_c, kD, kD * 2, 1, 64)) return cudaErrorInvalidValue;
-  if (!make_map_bf16_2d(&m.vc, vc, rows_c, kD, kD * 2, 1, 64)) return cudaErrorInvalidValue;
-  if (!make_map_bf16_2d(&m.kw, a.kw, (uint64_t)batch * a.ring, kD, kD * 2, 1, 64)) return cudaErrorInvalidValue;
-  if (!make_map_bf16_2d(&m.vw, a.vw, (uint64_t)batch * a.ring, kD, kD * 2, 1, 64)) return cudaErrorInvalidValue;
+  if (!make_map_bf16_2d(&m.kw, a.kw, (uint64_t)batch * a.ring, kD, kD * 2, kTile, 64)) return cudaErrorInvalidValue;
+  if (!make_map_bf16_2d(&m.vw, a.vw, (uint64_t)batch * a.ring, kD, kD * 2, kTile, 64)) return cudaErrorInvalidValue;
+  // Masked keys copy a row of their own source; with no compressed cache at all the
+  // compressed source is the window ring (row b*0 + 0), so that row is real memory.
   AttnArgs aa = a;
-  if (no_cache) aa.nc_cap = 0;   // compressed rows then index the ring map from row b*0
+  if (a.kc == nullptr || a.vc == nullptr || a.nc_cap <= 0) {
+    aa.kc = a.kw;
+    aa.vc = a.vw;
+    aa.nc_cap = 0;
+  }
   const int n_items = batch * a.T * a.nsplit;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

@@ -3,14 +3,15 @@
 //
 // One CTA per row, each thread holding EPT consecutive scores of the row in
 // registers as order-preserving uint32 keys (blocked layout: thread t owns
-// positions [t*EPT, (t+1)*EPT)).  The k-th largest key K* is found exactly
-// with three radix passes of 11, 11 and 10 bits.  The first pass, where most
-// keys share a few high digits, counts into 8 privatised histograms (two
-// 16-bit counters per word) that are summed afterwards; later passes only see
-// the keys that still match the prefix.  Because the layout is blocked, the
-// ordered output needs a single block-wide exclusive scan of per-thread
-// (greater-than, equal-to) counts; every thread then writes its selected
-// positions in ascending order, the lowest-index keys equal to K* first.
+// positions [t*EPT, (t+1)*EPT)).  A 12-bit radix pass (4096-bin shared
+// histogram) finds the bin that holds the k-th largest key; the keys of that
+// bin are compacted and, when there are at most 512 of them (the usual case),
+// ranked against each other by (key descending, position ascending), which
+// yields the exact k-th key K* and how many keys equal to it are taken.  Rows
+// where more keys share the bin take two further radix passes (12 and 8
+// bits).  Because the layout is blocked, the ordered output needs a single
+// block-wide exclusive scan of per-thread (greater-than, equal-to) counts;
+// every thread then writes its selected positions in ascending order.
 #pragma once
 #include "common.cuh"
 #include "topk.cuh"
@@ -18,15 +19,18 @@
 namespace hyb {
 
 constexpr int kRegEPT = 32;
+constexpr int kSelBins = 4096;       // 12-bit digits
+constexpr int kSelCand = 512;        // boundary-bin candidates resolved by ranking
 
 template <int THREADS>
 struct RegSelSmem {
-  uint32_t hist_w[8][1024];
-  uint32_t hist[2048];
+  uint32_t hist[kSelBins];
+  uint32_t cand_key[kSelCand];
+  int cand_pos[kSelCand];
   uint32_t warp_tot[THREADS / 32];
   uint32_t warp_off[THREADS / 32];
   uint32_t total;
-  uint32_t prefix, remaining;
+  uint32_t prefix, remaining, kth, need;
 };
 
 // Exclusive prefix sum over the CTA of one value per thread; `total` receives the sum.
@@ -58,28 +62,28 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, RegSelSmem<
   return sh.warp_off[warp] + incl - v;
 }
 
-// Finds the digit d (bins of width 2048 / THREADS per thread) such that
-// above(d) < rem <= above(d) + hist[d]; stores prefix |= d << shift, remaining.
+// Finds the digit d of `nbins` bins (each thread owns nbins / THREADS of them) with
+// above(d) < remaining <= above(d) + hist[d]; sets prefix |= d << shift and
+// remaining -= above(d).
 template <int THREADS>
-__device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift) {
-  constexpr int BPT = 2048 / THREADS;
-  uint32_t h[BPT], tot = 0;
-#pragma unroll
-  for (int e = 0; e < BPT; ++e) { h[e] = sh.hist[threadIdx.x * BPT + e]; tot += h[e]; }
+__device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift, int nbins) {
+  const int bpt = nbins / THREADS;
+  uint32_t tot = 0;
+  for (int e = 0; e < bpt; ++e) tot += sh.hist[threadIdx.x * bpt + e];
   const uint32_t rem = sh.remaining;
   const uint32_t prefix = sh.prefix;
   uint32_t total;
   const uint32_t before = block_exclusive_scan<THREADS>(tot, sh, total);
   uint32_t above = total - before - tot;    // keys in bins above this thread's range
   if (above < rem && rem <= above + tot) {
-#pragma unroll
-    for (int e = BPT - 1; e >= 0; --e) {
-      if (above + h[e] >= rem) {
-        sh.prefix = prefix | ((uint32_t)(threadIdx.x * BPT + e) << shift);
+    for (int e = bpt - 1; e >= 0; --e) {
+      const uint32_t h = sh.hist[threadIdx.x * bpt + e];
+      if (above + h >= rem) {
+        sh.prefix = prefix | ((uint32_t)(threadIdx.x * bpt + e) << shift);
         sh.remaining = rem - above;
         break;
       }
-      above += h[e];
+      above += h;
     }
   }
   __syncthreads();
@@ -88,7 +92,7 @@ __device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift) {
 template <int THREADS, typename Map>
 __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, int k_out, int* __restrict__ out,
                                Map map, RegSelSmem<THREADS>& sh) {
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x;
   if (n <= k) {
     for (int i = tid; i < k_out; i += THREADS) out[i] = i < n ? map(i) : -1;
     return;
@@ -107,43 +111,65 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
 #pragma unroll
     for (int e = 0; e < kRegEPT; ++e) key[e] = e < cnt ? score_key(scores[base + e]) : 0u;
   }
-  // ---- pass 0: bits 31..21, privatised histograms
-  for (int i = tid; i < 8 * 1024; i += THREADS) (&sh.hist_w[0][0])[i] = 0u;
+  // ---- pass 0: bits 31..20
+  for (int b = tid; b < kSelBins; b += THREADS) sh.hist[b] = 0u;
   if (tid == 0) { sh.prefix = 0; sh.remaining = (uint32_t)k; }
   __syncthreads();
-  uint32_t* hw = sh.hist_w[warp & 7];
 #pragma unroll
   for (int e = 0; e < kRegEPT; ++e)
-    if (e < cnt) {
-      const uint32_t d = key[e] >> 21;
-      atomicAdd(&hw[d >> 1], 1u << ((d & 1) * 16));
-    }
+    if (e < cnt) atomicAdd(&sh.hist[key[e] >> 20], 1u);
   __syncthreads();
-  for (int b = tid; b < 2048; b += THREADS) {
-    uint32_t s = 0;
+  find_digit<THREADS>(sh, 20, kSelBins);
+  const uint32_t prefix0 = sh.prefix, rem0 = sh.remaining;
+  // ---- keys in the boundary bin: rank them directly when there are few
+  uint32_t mine = 0;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) s += (sh.hist_w[w][b >> 1] >> ((b & 1) * 16)) & 0xFFFFu;
-    sh.hist[b] = s;
-  }
-  __syncthreads();
-  find_digit<THREADS>(sh, 21);
-  // ---- passes 1, 2: bits 20..10 and 9..0 of the keys that match the prefix
-  uint32_t mask = 0xFFE00000u;
-#pragma unroll 1
-  for (int pass = 1; pass < 3; ++pass) {
-    const int shift = pass == 1 ? 10 : 0;
-    const uint32_t dmask = pass == 1 ? 0x7FFu : 0x3FFu;
-    for (int b = tid; b < 2048; b += THREADS) sh.hist[b] = 0u;
-    __syncthreads();
-    const uint32_t prefix = sh.prefix;
+  for (int e = 0; e < kRegEPT; ++e) mine += (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) ? 1u : 0u;
+  uint32_t n_cand;
+  uint32_t slot = block_exclusive_scan<THREADS>(mine, sh, n_cand);
+  if (n_cand <= (uint32_t)kSelCand) {
 #pragma unroll
     for (int e = 0; e < kRegEPT; ++e)
-      if (e < cnt && (key[e] & mask) == prefix) atomicAdd(&sh.hist[(key[e] >> shift) & dmask], 1u);
+      if (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) {
+        sh.cand_key[slot] = key[e];
+        sh.cand_pos[slot] = base + e;
+        ++slot;
+      }
     __syncthreads();
-    find_digit<THREADS>(sh, shift);
-    mask |= dmask << shift;
+    // rank by (key descending, position ascending); the candidate of rank rem0-1 is K*
+    for (uint32_t c = tid; c < n_cand; c += THREADS) {
+      const uint32_t kc = sh.cand_key[c];
+      const int pc = sh.cand_pos[c];
+      uint32_t rank = 0, greater = 0;
+      for (uint32_t j = 0; j < n_cand; ++j) {
+        const uint32_t kj = sh.cand_key[j];
+        greater += kj > kc;
+        rank += kj > kc || (kj == kc && sh.cand_pos[j] < pc);
+      }
+      if (rank == rem0 - 1) { sh.kth = kc; sh.need = rem0 - greater; }
+    }
+    __syncthreads();
+  } else {
+    // ---- many keys share the first digit: two more radix passes
+    uint32_t mask = 0xFFF00000u;
+#pragma unroll 1
+    for (int pass = 1; pass < 3; ++pass) {
+      const int shift = pass == 1 ? 8 : 0;
+      const uint32_t dmask = pass == 1 ? 0xFFFu : 0xFFu;
+      for (int b = tid; b < kSelBins; b += THREADS) sh.hist[b] = 0u;
+      __syncthreads();
+      const uint32_t prefix = sh.prefix;
+#pragma unroll
+      for (int e = 0; e < kRegEPT; ++e)
+        if (e < cnt && (key[e] & mask) == prefix) atomicAdd(&sh.hist[(key[e] >> shift) & dmask], 1u);
+      __syncthreads();
+      find_digit<THREADS>(sh, shift, pass == 1 ? kSelBins : 256 < THREADS ? THREADS : 256);
+      mask |= dmask << shift;
+    }
+    if (tid == 0) { sh.kth = sh.prefix; sh.need = sh.remaining; }
+    __syncthreads();
   }
-  const uint32_t kth = sh.prefix, need = sh.remaining;
+  const uint32_t kth = sh.kth, need = sh.need;
   // ---- ordered output
   uint32_t gt = 0, eq = 0;
 #pragma unroll
