@@ -37,7 +37,9 @@
 // are rescaled; otherwise probabilities are taken against the stale maximum
 // (they stay below 2^8).  P^T is written as a bf16 MN-major operand in shared
 // memory, one 128-byte row per key.  Row sums are reduced across key lanes once
-// per query.  A work item is a query or, for split-KV decode, a tile-aligned
+// per query.  The normalised bf16 output tile o[h][d] is staged in shared memory
+// and written to global memory by one bulk copy on the TMA engine; keys masked
+// out (indexer padding) are zero-filled by the producers without a global read.  A work item is a query or, for split-KV decode, a tile-aligned
 // slice of its keys; slices write partial (o, lse) pairs that attn_merge combines.
 #pragma once
 #include "attn.cuh"
@@ -57,7 +59,8 @@ constexpr int kProdLanes = kProdWarps * 32;
 constexpr int kQBytes = kH * kD * 2;                    // 16 KB, two 64-column sub-tiles
 constexpr int kKVBytes = kTile * kD * 2;                // 32 KB, two 64-column sub-tiles
 constexpr int kPBytes = kTile * kH * 2;                 // 16 KB
-constexpr int kSmem = kQSt * kQBytes + kKSt * kKVBytes + kVSt * kKVBytes + kPSt * kPBytes + 1024;
+constexpr int kOBytes = kH * kD * 2;                    // 16 KB bf16 output tile, [h][d]
+constexpr int kSmem = kQSt * kQBytes + kKSt * kKVBytes + kVSt * kKVBytes + kPSt * kPBytes + kOBytes + 1024;
 constexpr uint32_t kSCols = kGT * kH;                   // 192 columns per S^T buffer
 constexpr uint32_t kOCol = 2 * kSCols;                  // O^T buffers at 384 and 448
 constexpr float kRescaleThreshold = 8.f;                // base-2 units
@@ -196,6 +199,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   uint8_t* sK = sQ + kQSt * kQBytes;
   uint8_t* sV = sK + kKSt * kKVBytes;
   uint8_t* sP = sV + kVSt * kKVBytes;
+  uint8_t* sO = sP + kPSt * kPBytes;
 
   __shared__ uint64_t q_full[kQSt], q_empty[kQSt], k_full[kKSt], k_empty[kKSt], v_full[kVSt], v_empty[kVSt];
   __shared__ uint64_t s_full[2], s_free[2], p_full[kPSt], p_empty[kPSt], o_full[2], o_ready[2];
@@ -311,7 +315,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
             }
           } else {
             // gathered rows: 16-byte cp.async per lane, lane-consecutive chunks of a
-            // 256-byte row, written with the 128-byte swizzle the MMA descriptors expect
+            // 256-byte row, written with the 128-byte swizzle the MMA descriptors expect;
+            // a masked key's row is zero-filled without reading global memory
             const int safe = tbl.safe[slot][j];
             const bool win = tbl.win[slot][j] != 0;
             const char* src = static_cast<const char*>(is_k ? (win ? a.kw : a.kc) : (win ? a.vw : a.vc));
@@ -322,10 +327,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
               const int q = i * kProdLanes + plane;
               if (q < kTile * 16) {
                 const int r = q >> 4, c = (q >> 3) & 1, ch = q & 7;
-                int rw = trow[r];
-                rw = rw >= 0 ? rw : safe;
-                cp_async16(dbase + c * (kKVBytes / 2) + r * 128 + ((ch ^ (r & 7)) << 4),
-                           src + (size_t)rw * (kD * 2) + c * 128 + ch * 16);
+                const int rw = trow[r];
+                cp_async16_zfill(dbase + c * (kKVBytes / 2) + r * 128 + ((ch ^ (r & 7)) << 4),
+                                 src + (size_t)(rw >= 0 ? rw : safe) * (kD * 2) + c * 128 + ch * 16, rw >= 0 ? 16u : 0u);
               }
             }
           }
@@ -559,6 +563,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         fence_after_sync();
         warp_xsum32(lp, lane);
         red[hf][quad][lane] = lp[0];
+        if (warp == 8 && lane == 0) bulk_wait_read_all();   // the previous item's output tile has left sO
         named_sync_softmax();
         if (quad == 0) {
           const int h = hf * 32 + lane;
@@ -572,19 +577,36 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         uint32_t v[32];
         tmem_ld32(lane_addr + kOCol + ob * kH + hf * 32, v);
         tmem_wait_ld();
+        if (final_out) {
+          // o[h][d] is staged in shared memory and leaves as one 16 KB bulk copy on
+          // the TMA engine, off the load/store path the producers' gathers occupy
+          bf16* so = reinterpret_cast<bf16*>(sO);
+#pragma unroll 8
+          for (int e = 0; e < 32; ++e) {
+            const int h = hf * 32 + e;
+            const float l = l_fin[h];
+            so[h * kD + kk] = __float2bfloat16_rn(l > 0.f ? __uint_as_float(v[e]) / l : 0.f);
+          }
+          fence_proxy_async_smem();
+          named_sync_softmax();
+          if (warp == 8 && lane == 0) {
+            bulk_store_s2g(static_cast<bf16*>(a.o) + prow * kD, smem_u32(sO), kOBytes);
+            bulk_commit();
+          }
+        } else {
 #pragma unroll 4
-        for (int e = 0; e < 32; ++e) {
-          const int h = hf * 32 + e;
-          const float l = l_fin[h];
-          const float o = l > 0.f ? __uint_as_float(v[e]) / l : 0.f;
-          if (final_out) store_f((bf16*)a.o + (prow + h) * kD + kk, o);
-          else a.part_o[(prow + h) * kD + kk] = o;
+          for (int e = 0; e < 32; ++e) {
+            const int h = hf * 32 + e;
+            const float l = l_fin[h];
+            a.part_o[(prow + h) * kD + kk] = l > 0.f ? __uint_as_float(v[e]) / l : 0.f;
+          }
         }
         fence_before_sync();
         named_sync_softmax();   // l_fin / m_run are rewritten by the next item
       }
       ++n;
     }
+    if (warp == 8 && lane == 0) bulk_wait_all();
   }
   fence_before_sync();
   __syncthreads();
@@ -595,9 +617,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
 }  // namespace attn_tc
 
 inline bool attn_tc_supported(int H, int D, const void* q, const void* kc, const void* vc, const void* kw,
-                              const void* vw) {
+                              const void* vw, const void* o) {
   auto al = [](const void* p) { return p == nullptr || reinterpret_cast<uintptr_t>(p) % 16 == 0; };
-  return H == attn_tc::kH && D == attn_tc::kD && al(q) && al(kc) && al(vc) && al(kw) && al(vw);
+  return H == attn_tc::kH && D == attn_tc::kD && al(q) && al(kc) && al(vc) && al(kw) && al(vw) && al(o);
 }
 
 // Launches the tensor-core attention for all batch*T queries (nsplit slices each).

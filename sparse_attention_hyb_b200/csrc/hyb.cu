@@ -309,7 +309,7 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const
     return HYB_ERR_INVALID_ARG;
   if (batch == 0 || T == 0) return HYB_OK;
   if (!q || !q_pos || !kw || !vw || !o || ((nc > 0) && (!kc || !vc))) return HYB_ERR_INVALID_ARG;
-  if (!attn_ffma_supported(H, D) && !(dtype == HYB_DTYPE_BF16 && attn_tc_supported(H, D, q, kc, vc, kw, vw)))
+  if (!attn_ffma_supported(H, D) && !(dtype == HYB_DTYPE_BF16 && attn_tc_supported(H, D, q, kc, vc, kw, vw, o)))
     return HYB_ERR_UNSUPPORTED;
   const int n_keys = (idx ? k : nc) + W;
   const int ns = attn_splits(mode, batch, T, n_keys);
@@ -328,7 +328,7 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const
     if ((e = launch_attn_ffma<float>(a, batch, s)) != cudaSuccess) return HYB_ERR_CUDA;
     if (ns > 1) { attn_merge_kernel<float><<<dim3(batch * T, H), 128, 0, s>>>(a); count_launch(); }
   } else {
-    if (attn_tc_supported(H, D, q, kc, vc, kw, vw))
+    if (attn_tc_supported(H, D, q, kc, vc, kw, vw, o))
       e = launch_attn_tc(a, batch, s);
     else
       e = launch_attn_ffma<bf16>(a, batch, s);
