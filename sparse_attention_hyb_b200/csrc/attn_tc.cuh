@@ -208,7 +208,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   __shared__ float red[2][4][32];
-  __shared__ float m_run[kH], m_use[kH], alpha_s[kH], l_fin[kH];
+  __shared__ float m_run[kH], alpha_s[kH];
+  __shared__ __align__(16) float m_use[kH];
+  __shared__ __align__(16) float l_inv[kH];   // 1 / row sum, 0 for a head with no key
   __shared__ int resc_flag[2];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -533,13 +535,18 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           uint32_t pk[16];
           const bool valid = (vmask >> j) & 1u;
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float p0 = valid ? ex2_approx(fmaf(__uint_as_float(v[e]), c2, -mu[e])) : 0.f;
-            const float p1 = valid ? ex2_approx(fmaf(__uint_as_float(v[e + 1]), c2, -mu[e + 1])) : 0.f;
-            lp[e] += p0;
-            lp[e + 1] += p1;
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-            pk[e / 2] = *reinterpret_cast<uint32_t*>(&b2);
+          for (int e = 0; e < 32; e += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(mu + e);
+            const float m[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+            for (int i = 0; i < 4; i += 2) {
+              const float p0 = valid ? ex2_approx(fmaf(__uint_as_float(v[e + i]), c2, -m[i])) : 0.f;
+              const float p1 = valid ? ex2_approx(fmaf(__uint_as_float(v[e + i + 1]), c2, -m[i + 1])) : 0.f;
+              lp[e + i] += p0;
+              lp[e + i + 1] += p1;
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+              pk[(e + i) / 2] = *reinterpret_cast<uint32_t*>(&b2);
+            }
           }
           uint8_t* prow_s = sP + ps * kPBytes + kk * 128;
 #pragma unroll
@@ -568,7 +575,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         if (quad == 0) {
           const int h = hf * 32 + lane;
           const float l = red[hf][0][lane] + red[hf][1][lane] + red[hf][2][lane] + red[hf][3][lane];
-          l_fin[h] = l;
+          l_inv[h] = l > 0.f ? 1.f / l : 0.f;
           const float lse = l > 0.f ? m_run[h] * 0.6931471805599453f + logf(l) : -INFINITY;
           if (final_out) { if (a.lse) a.lse[prow + h] = lse; }
           else a.part_lse[prow + h] = lse;
@@ -581,11 +588,12 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           // o[h][d] is staged in shared memory and leaves as one 16 KB bulk copy on
           // the TMA engine, off the load/store path the producers' gathers occupy
           bf16* so = reinterpret_cast<bf16*>(sO);
-#pragma unroll 8
-          for (int e = 0; e < 32; ++e) {
-            const int h = hf * 32 + e;
-            const float l = l_fin[h];
-            so[h * kD + kk] = __float2bfloat16_rn(l > 0.f ? __uint_as_float(v[e]) / l : 0.f);
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 r4 = *reinterpret_cast<const float4*>(l_inv + hf * 32 + e);
+            const float r[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) so[(hf * 32 + e + i) * kD + kk] = __float2bfloat16_rn(__uint_as_float(v[e + i]) * r[i]);
           }
           fence_proxy_async_smem();
           named_sync_softmax();
@@ -597,12 +605,11 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
 #pragma unroll 4
           for (int e = 0; e < 32; ++e) {
             const int h = hf * 32 + e;
-            const float l = l_fin[h];
-            a.part_o[(prow + h) * kD + kk] = l > 0.f ? __uint_as_float(v[e]) / l : 0.f;
+            a.part_o[(prow + h) * kD + kk] = __uint_as_float(v[e]) * l_inv[h];
           }
         }
         fence_before_sync();
-        named_sync_softmax();   // l_fin / m_run are rewritten by the next item
+        named_sync_softmax();   // l_inv / m_run are rewritten by the next item
       }
       ++n;
     }
