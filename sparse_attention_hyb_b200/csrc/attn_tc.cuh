@@ -343,75 +343,139 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     cp_async_wait<0>();
   } else {
     // ======================================================== MMA issuer
+    // Two in-order streams, scheduled by readiness instead of program order: the
+    // S^T tiles of the groups (K tiles as they land) and the O^T += V^T P^T tiles
+    // of groups whose probabilities are being produced.  Neither waits for the
+    // other, so the last O^T update of a query does not wait for the next
+    // query's K tiles, and S^T of the next group overlaps the current softmax.
     if (lane == 0) {
       constexpr uint32_t idesc1 = idesc_bf16_f32(128, kH, false, false);
       constexpr uint32_t idesc2 = idesc_bf16_f32(128, kH, true, true);
-      uint32_t G = 0, n = 0, kt = 0, vt = 0, pt = 0;
-      uint32_t ordy[2] = {0, 0};
-      PendingPV pend{0, 0, 0, 0};
-      bool ok = true;
-      auto issue_pv = [&](const PendingPV& pv) {
-        if (!ok) return;
-        ok = mbar_wait(&o_ready[pv.ob], full_par(ordy[pv.ob], 1), &abort_flag);
-        ++ordy[pv.ob];
-        for (int j = 0; j < pv.ntiles && ok; ++j) {
-          const int vs = vt % kVSt, ps = pt % kPSt;
-          ok = mbar_wait(&v_full[vs], full_par(vt, kVSt), &abort_flag) &&
-               mbar_wait(&p_full[ps], full_par(pt, kPSt), &abort_flag);
-          if (!ok) break;
-          fence_after_sync();
-          fence_async_shared();
-          const uint32_t vbase = smem_u32(sV + vs * kKVBytes);
-          const uint32_t pbase = smem_u32(sP + ps * kPBytes);
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_f16_ss(tmem + kOCol + pv.ob * kH, desc_mnmajor_sw128(vbase + kk * 2048, kKVBytes / 2),
-                       desc_mnmajor_sw128(pbase + kk * 2048, 0), idesc2, (pv.first && j == 0 && kk == 0) ? 0u : 1u);
-          mma_commit(&v_empty[vs]);
-          mma_commit(&p_empty[ps]);
-          ++vt;
-          ++pt;
-        }
-        mma_commit(&o_full[pv.ob]);
-      };
-      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
-        Item it;
-        it.init(a, w);
-        if (it.n_tiles() == 0) continue;
-        const int qb = n % kQSt, ob = n % 2;
-        bool first = true;
-        for (int g0 = it.tile_beg; g0 < it.tile_end && ok; g0 += kGT, ++G) {
-          const int nt = min(kGT, it.tile_end - g0);
-          const bool last = g0 + kGT >= it.tile_end;
-          const int sb = G % 2;
-          ok = mbar_wait(&s_free[sb], empty_par(G, 2), &abort_flag);
-          if (ok && first) ok = mbar_wait(&q_full[qb], full_par(n, kQSt), &abort_flag);
-          for (int j = 0; j < nt && ok; ++j, ++kt) {
-            const int ks = kt % kKSt;
-            ok = mbar_wait(&k_full[ks], full_par(kt, kKSt), &abort_flag);
-            if (!ok) break;
-            fence_after_sync();
-            fence_async_shared();
-            const uint32_t d = tmem + sb * kSCols + j * kH;
-            const uint32_t kbase = smem_u32(sK + ks * kKVBytes);
-            const uint32_t qbase = smem_u32(sQ + qb * kQBytes);
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_f16_ss(d, desc_kmajor_sw128(kbase + c * (kKVBytes / 2) + kk * 32),
-                           desc_kmajor_sw128(qbase + c * (kQBytes / 2) + kk * 32), idesc1, (c | kk) != 0);
-            mma_commit(&k_empty[ks]);
+      constexpr int kRing = 4;
+      // S stream
+      Item s_it;
+      int s_w = blockIdx.x, s_g0 = 0, s_nt = 0, s_j = 0;
+      bool s_have = false, s_first = true, s_open = false;
+      uint32_t Gs = 0, ns = 0, kt = 0;
+      // PV stream: groups whose S^T has been issued, oldest first
+      PendingPV ring[kRing];
+      int ph = 0, pc = 0, p_j = 0;
+      bool p_open = false;
+      uint32_t vt = 0, pt = 0, ordy[2] = {0, 0};
+      uint32_t idle = 0;
+      unsigned long long idle_t0 = 0;
+      for (;;) {
+        bool prog = false;
+        if (!s_have) {
+          for (; s_w < n_items; s_w += gridDim.x) {
+            s_it.init(a, s_w);
+            if (s_it.n_tiles() > 0) break;
           }
-          mma_commit(&s_full[sb]);
-          if (last) mma_commit(&q_empty[qb]);
-          if (pend.valid) issue_pv(pend);
-          pend = PendingPV{1, ob, nt, first ? 1 : 0};
-          first = false;
+          if (s_w < n_items) {
+            s_have = true;
+            s_first = true;
+            s_open = false;
+            s_g0 = s_it.tile_beg;
+          }
         }
-        ++n;
+        if (s_have && pc < kRing) {
+          const int sb = Gs % 2, qb = ns % kQSt;
+          if (!s_open && mbar_try_wait(&s_free[sb], empty_par(Gs, 2)) &&
+              (!s_first || mbar_try_wait(&q_full[qb], full_par(ns, kQSt)))) {
+            s_open = true;
+            s_nt = min(kGT, s_it.tile_end - s_g0);
+            s_j = 0;
+          }
+          if (s_open) {
+            while (s_j < s_nt) {
+              const int ks = kt % kKSt;
+              if (!mbar_try_wait(&k_full[ks], full_par(kt, kKSt))) break;
+              fence_after_sync();
+              fence_async_shared();
+              const uint32_t d = tmem + sb * kSCols + s_j * kH;
+              const uint32_t kbase = smem_u32(sK + ks * kKVBytes);
+              const uint32_t qbase = smem_u32(sQ + qb * kQBytes);
+#pragma unroll
+              for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_f16_ss(d, desc_kmajor_sw128(kbase + c * (kKVBytes / 2) + kk * 32),
+                             desc_kmajor_sw128(qbase + c * (kQBytes / 2) + kk * 32), idesc1, (c | kk) != 0);
+              mma_commit(&k_empty[ks]);
+              ++kt;
+              ++s_j;
+              prog = true;
+            }
+            if (s_j == s_nt) {
+              const bool last = s_g0 + kGT >= s_it.tile_end;
+              mma_commit(&s_full[sb]);
+              if (last) mma_commit(&q_empty[qb]);
+              ring[(ph + pc) % kRing] = PendingPV{1, static_cast<int>(ns % 2), s_nt, s_first ? 1 : 0};
+              ++pc;
+              ++Gs;
+              s_first = false;
+              s_open = false;
+              s_g0 += kGT;
+              if (last) {
+                s_have = false;
+                ++ns;
+                s_w += gridDim.x;
+              }
+              prog = true;
+            }
+          }
+        }
+        if (pc > 0) {
+          const PendingPV pv = ring[ph];
+          if (!p_open && mbar_try_wait(&o_ready[pv.ob], full_par(ordy[pv.ob], 1))) {
+            ++ordy[pv.ob];
+            p_open = true;
+            p_j = 0;
+            prog = true;
+          }
+          if (p_open) {
+            while (p_j < pv.ntiles) {
+              const int vs = vt % kVSt, ps = pt % kPSt;
+              if (!mbar_try_wait(&v_full[vs], full_par(vt, kVSt)) || !mbar_try_wait(&p_full[ps], full_par(pt, kPSt))) break;
+              fence_after_sync();
+              fence_async_shared();
+              const uint32_t vbase = smem_u32(sV + vs * kKVBytes);
+              const uint32_t pbase = smem_u32(sP + ps * kPBytes);
+#pragma unroll
+              for (int kk = 0; kk < kTile / 16; ++kk)
+                mma_f16_ss(tmem + kOCol + pv.ob * kH, desc_mnmajor_sw128(vbase + kk * 2048, kKVBytes / 2),
+                           desc_mnmajor_sw128(pbase + kk * 2048, 0), idesc2, (pv.first && p_j == 0 && kk == 0) ? 0u : 1u);
+              mma_commit(&v_empty[vs]);
+              mma_commit(&p_empty[ps]);
+              ++vt;
+              ++pt;
+              ++p_j;
+              prog = true;
+            }
+            if (p_j == pv.ntiles) {
+              mma_commit(&o_full[pv.ob]);
+              p_open = false;
+              ph = (ph + 1) % kRing;
+              --pc;
+              prog = true;
+            }
+          }
+        }
+        if (!s_have && s_w >= n_items && pc == 0) break;
+        if (prog) {
+          idle = 0;
+        } else if ((++idle & 63u) == 0) {   // no progress: check the abort flag and the time limit
+          if (abort_flag) break;
+          const unsigned long long now = globaltimer();
+          if (idle == 64) {
+            idle_t0 = now;
+          } else if (now - idle_t0 > kWaitNs) {
+            abort_flag = 1;
+            report(HYB_ERR_TIMEOUT);
+            break;
+          }
+        }
       }
-      if (pend.valid) issue_pv(pend);
       mma_commit(&mma_done);
       const unsigned long long t0 = globaltimer();
       while (!mbar_try_wait(&mma_done, 0) && globaltimer() - t0 < kWaitNs) {}
