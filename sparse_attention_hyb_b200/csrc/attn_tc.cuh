@@ -52,7 +52,7 @@ namespace attn_tc {
 
 constexpr int kH = 64, kD = 128, kTile = 128;
 constexpr int kGT = 3;                                  // tiles per group
-constexpr int kQSt = 2, kKSt = 2, kVSt = 2, kPSt = 2, kTbl = 4;
+constexpr int kQSt = 2, kKSt = 2, kVSt = 2, kPSt = 2, kTbl = 8;
 constexpr int kThreads = 512;
 constexpr int kProdWarps = 3;                           // per tensor (K, V)
 constexpr int kProdLanes = kProdWarps * 32;
@@ -103,19 +103,22 @@ struct Item {
   __device__ int n_tiles() const { return tile_end - tile_beg; }
 };
 
-// Source of key kk of a tile: entry index (compressed) or ring slot (window);
-// -1 for padding / invalid keys.  Reports indices outside the visible range.
-__device__ __forceinline__ int key_source(const AttnArgs& a, const KeyList& kl, int tile, int kk) {
+// Indexer entry behind key kk of compressed tile `tile` (the dense range when
+// there is no indexer); -1 for window tiles and padding.  A pure load, so a
+// group's loads can all be in flight together.
+__device__ __forceinline__ int key_entry(const AttnArgs& a, const KeyList& kl, int tile, int kk) {
+  const int u = tile * kTile + kk;
+  if (tile >= kl.comp_tiles || u >= kl.n_comp) return -1;
+  return a.idx ? __ldg(a.idx + (size_t)kl.row * a.k + u) : u;
+}
+
+// Source of key kk of a tile: entry index (compressed, from its entry e) or ring
+// slot (window); -1 for padding / masked keys, -2 for an entry outside the
+// visible range.
+__device__ __forceinline__ int key_source(const AttnArgs& a, const KeyList& kl, int tile, int kk, int e) {
   if (tile < kl.comp_tiles) {
-    const int u = tile * kTile + kk;
-    if (u >= kl.n_comp) return -1;
-    const int j = a.idx ? __ldg(a.idx + (size_t)kl.row * a.k + u) : u;
-    if (j < 0) return -1;
-    if (j >= kl.vis) {
-      report(HYB_ERR_DEVICE_CHECK);
-      return -1;
-    }
-    return j;
+    if (e < 0) return -1;
+    return e < kl.vis ? e : -2;
   }
   const int u = (tile - kl.comp_tiles) * kTile + kk;
   if (u >= kl.n_win) return -1;
@@ -241,28 +244,68 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
   if (warp == 1) {
     // ======================================================== key tables and Q
-    uint32_t G = 0, n = 0;
+    // Q tiles are queued and issued by lane 0 whenever their slot is free, so
+    // building tables never waits for a Q slot.
+    constexpr int kQQ = 16;                 // queued Q loads (>= items a full table ring can span)
+    int qrow[kQQ];
+    uint32_t G = 0, n = 0, q_next = 0;
+    auto service_q = [&]() {
+      if (lane != 0) return;
+      while (q_next < n && mbar_try_wait(&q_empty[q_next % kQSt], empty_par(q_next, kQSt))) {
+        const int qb = q_next % kQSt;
+        mbar_expect_tx(&q_full[qb], kQBytes);
+        for (int c = 0; c < 2; ++c)
+          tma_load_2d(sQ + qb * kQBytes + c * (kQBytes / 2), &maps.q, &q_full[qb], c * 64, qrow[q_next % kQQ] * kH);
+        ++q_next;
+      }
+    };
+    // Polls `bar` while serving the Q queue; false on abort or time-out.
+    auto wait_serving = [&](uint64_t* bar, uint32_t par) {
+      const unsigned long long t0 = globaltimer();
+      for (uint32_t it = 0;; ++it) {
+        service_q();
+        if (mbar_try_wait(bar, par)) return true;
+        if ((it & 63u) == 63u) {
+          if (abort_flag) return false;
+          if (globaltimer() - t0 > kWaitNs) {
+            abort_flag = 1;
+            report(HYB_ERR_TIMEOUT);
+            return false;
+          }
+        }
+      }
+    };
     for (int w = blockIdx.x; w < n_items && !abort_flag; w += gridDim.x) {
       Item it;
       it.init(a, w);
       if (it.n_tiles() == 0) continue;
       const int b = it.kl.row / a.T;
-      const int qb = n % kQSt;
-      if (lane == 0 && mbar_wait(&q_empty[qb], empty_par(n, kQSt), &abort_flag)) {
-        mbar_expect_tx(&q_full[qb], kQBytes);
-        for (int c = 0; c < 2; ++c)
-          tma_load_2d(sQ + qb * kQBytes + c * (kQBytes / 2), &maps.q, &q_full[qb], c * 64, it.kl.row * kH);
+      if (lane == 0) {   // (q_next is lane 0's; the queue cannot fill while the table ring holds fewer groups)
+        if (n - q_next >= kQQ && wait_serving(&q_empty[q_next % kQSt], empty_par(q_next, kQSt))) service_q();
+        qrow[n % kQQ] = it.kl.row;
       }
       ++n;
+      service_q();
       for (int g0 = it.tile_beg; g0 < it.tile_end; g0 += kGT, ++G) {
         const int nt = min(kGT, it.tile_end - g0);
         const int slot = G % kTbl;
-        if (!mbar_wait(&t_empty[slot], empty_par(G, kTbl), &abort_flag)) break;
+        // the group's indexer loads are issued before the wait for its table slot
         int src[kGT][4];
 #pragma unroll
         for (int j = 0; j < kGT; ++j)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) src[j][i] = j < nt ? key_source(a, it.kl, g0 + j, lane + 32 * i) : -1;
+          for (int i = 0; i < 4; ++i) src[j][i] = j < nt ? key_entry(a, it.kl, g0 + j, lane + 32 * i) : -1;
+        if (!wait_serving(&t_empty[slot], empty_par(G, kTbl))) break;
+        bool bad = false;
+#pragma unroll
+        for (int j = 0; j < kGT; ++j)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int sj = j < nt ? key_source(a, it.kl, g0 + j, lane + 32 * i, src[j][i]) : -1;
+            bad |= sj == -2;
+            src[j][i] = sj < 0 ? -1 : sj;
+          }
+        if (bad) report(HYB_ERR_DEVICE_CHECK);
 #pragma unroll
         for (int j = 0; j < kGT; ++j) {
           if (j >= nt) break;
@@ -282,6 +325,16 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           }
         }
         mbar_arrive(&t_full[slot]);
+      }
+    }
+    if (lane == 0) {   // issue the Q tiles still queued
+      const unsigned long long t0 = globaltimer();
+      while (q_next < n && !abort_flag) {
+        service_q();
+        if (globaltimer() - t0 > kWaitNs) {
+          abort_flag = 1;
+          report(HYB_ERR_TIMEOUT);
+        }
       }
     }
   } else if (warp >= 2) {
