@@ -465,7 +465,8 @@ def run_ours(args, world, rank, local):
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{pk_src} bf16 burst", "flops_per_launch": res["attn_flops"]},
         "gpu_launches": res["launches"],
-        "e2e": {"value": world * w.T / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": None if math.isnan(e2e_ms) else world * w.T / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "clocks": clocks,
         "decode": decode,
