@@ -1,17 +1,17 @@
 // Top-k selection, register-resident variant (HISA write-up, section 01: keep
 // the k highest-scoring entries; ties go to the lower index).
 //
-// One CTA per row, each thread holding EPT consecutive scores of the row in
-// registers as order-preserving uint32 keys (blocked layout: thread t owns
-// positions [t*EPT, (t+1)*EPT)).  A 12-bit radix pass (4096-bin shared
-// histogram) finds the bin that holds the k-th largest key; the keys of that
-// bin are compacted and, when there are at most 512 of them (the usual case),
-// ranked against each other by (key descending, position ascending), which
-// yields the exact k-th key K* and how many keys equal to it are taken.  Rows
-// where more keys share the bin take two further radix passes (12 and 8
-// bits).  Because the layout is blocked, the ordered output needs a single
-// block-wide exclusive scan of per-thread (greater-than, equal-to) counts;
-// every thread then writes its selected positions in ascending order.
+// One CTA per row, each thread holding EPT (8, 16 or 32, chosen per row from its
+// length) consecutive scores of the row in registers as order-preserving uint32
+// keys (blocked layout: thread t owns positions [t*EPT, (t+1)*EPT)).  A 12-bit
+// radix pass (4096-bin shared histogram) finds the bin that holds the k-th
+// largest key.  The keys of that bin are compacted into shared memory (normally
+// a few hundred at most) and two more radix passes over them alone (12 and 8
+// bits) give the exact k-th key K* and how many keys equal to it are taken;
+// rows where more keys share the bin run those passes over the registers.
+// Because the layout is blocked, the ordered output needs a single block-wide
+// exclusive scan of per-thread (greater-than, equal-to) counts; every thread
+// then writes its selected positions in ascending order.
 #pragma once
 #include "common.cuh"
 #include "topk.cuh"
@@ -24,9 +24,8 @@ constexpr int kSelCand = 512;        // boundary-bin candidates resolved by rank
 
 template <int THREADS>
 struct RegSelSmem {
-  uint32_t hist[kSelBins];
+  alignas(16) uint32_t hist[kSelBins];
   uint32_t cand_key[kSelCand];
-  int cand_pos[kSelCand];
   uint32_t warp_tot[THREADS / 32];
   uint32_t warp_off[THREADS / 32];
   uint32_t total;
@@ -69,7 +68,15 @@ template <int THREADS>
 __device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift, int nbins) {
   const int bpt = nbins / THREADS;
   uint32_t tot = 0;
-  for (int e = 0; e < bpt; ++e) tot += sh.hist[threadIdx.x * bpt + e];
+  if (bpt % 4 == 0) {
+    const uint4* h4 = reinterpret_cast<const uint4*>(sh.hist + threadIdx.x * bpt);
+    for (int e = 0; e < bpt / 4; ++e) {
+      const uint4 v = h4[e];
+      tot += v.x + v.y + v.z + v.w;
+    }
+  } else {
+    for (int e = 0; e < bpt; ++e) tot += sh.hist[threadIdx.x * bpt + e];
+  }
   const uint32_t rem = sh.remaining;
   const uint32_t prefix = sh.prefix;
   uint32_t total;
@@ -89,7 +96,13 @@ __device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift, i
   __syncthreads();
 }
 
-template <int THREADS, typename Map>
+// Zeroes the first `nbins` histogram bins (a multiple of 4).
+template <int THREADS>
+__device__ __forceinline__ void zero_hist(RegSelSmem<THREADS>& sh, int nbins) {
+  for (int b = threadIdx.x; b < nbins / 4; b += THREADS) reinterpret_cast<uint4*>(sh.hist)[b] = make_uint4(0, 0, 0, 0);
+}
+
+template <int THREADS, int EPT, typename Map>
 __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, int k_out, int* __restrict__ out,
                                Map map, RegSelSmem<THREADS>& sh) {
   const int tid = threadIdx.x;
@@ -98,88 +111,83 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
     return;
   }
   for (int i = k + tid; i < k_out; i += THREADS) out[i] = -1;
-  const int base = tid * kRegEPT;
-  const int cnt = n - base < 0 ? 0 : (n - base > kRegEPT ? kRegEPT : n - base);
-  uint32_t key[kRegEPT];
-  if (cnt == kRegEPT && (reinterpret_cast<uintptr_t>(scores + base) & 15) == 0) {
+  const int base = tid * EPT;
+  const int cnt = n - base < 0 ? 0 : (n - base > EPT ? EPT : n - base);
+  uint32_t key[EPT];
+  if (cnt == EPT && (reinterpret_cast<uintptr_t>(scores + base) & 15) == 0) {
 #pragma unroll
-    for (int e = 0; e < kRegEPT; e += 4) {
+    for (int e = 0; e < EPT; e += 4) {
       const float4 f = *reinterpret_cast<const float4*>(scores + base + e);
       key[e] = score_key(f.x); key[e + 1] = score_key(f.y); key[e + 2] = score_key(f.z); key[e + 3] = score_key(f.w);
     }
   } else {
 #pragma unroll
-    for (int e = 0; e < kRegEPT; ++e) key[e] = e < cnt ? score_key(scores[base + e]) : 0u;
+    for (int e = 0; e < EPT; ++e) key[e] = e < cnt ? score_key(scores[base + e]) : 0u;
   }
+  constexpr int kLastBins = 256 < THREADS ? THREADS : 256;   // 8-bit pass, at least one bin per thread
   // ---- pass 0: bits 31..20
-  for (int b = tid; b < kSelBins; b += THREADS) sh.hist[b] = 0u;
+  zero_hist<THREADS>(sh, kSelBins);
   if (tid == 0) { sh.prefix = 0; sh.remaining = (uint32_t)k; }
   __syncthreads();
 #pragma unroll
-  for (int e = 0; e < kRegEPT; ++e)
+  for (int e = 0; e < EPT; ++e)
     if (e < cnt) atomicAdd(&sh.hist[key[e] >> 20], 1u);
   __syncthreads();
   find_digit<THREADS>(sh, 20, kSelBins);
-  const uint32_t prefix0 = sh.prefix, rem0 = sh.remaining;
-  // ---- keys in the boundary bin: rank them directly when there are few
+  const uint32_t prefix0 = sh.prefix;
+  // ---- the boundary bin's keys
   uint32_t mine = 0;
 #pragma unroll
-  for (int e = 0; e < kRegEPT; ++e) mine += (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) ? 1u : 0u;
+  for (int e = 0; e < EPT; ++e) mine += (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) ? 1u : 0u;
   uint32_t n_cand;
   uint32_t slot = block_exclusive_scan<THREADS>(mine, sh, n_cand);
+  zero_hist<THREADS>(sh, kSelBins);
   if (n_cand <= (uint32_t)kSelCand) {
+    // few: compact them and resolve the low 20 bits over the candidates alone
 #pragma unroll
-    for (int e = 0; e < kRegEPT; ++e)
-      if (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) {
-        sh.cand_key[slot] = key[e];
-        sh.cand_pos[slot] = base + e;
-        ++slot;
-      }
+    for (int e = 0; e < EPT; ++e)
+      if (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) sh.cand_key[slot++] = key[e];
     __syncthreads();
-    // rank by (key descending, position ascending); the candidate of rank rem0-1 is K*
+    for (uint32_t c = tid; c < n_cand; c += THREADS) atomicAdd(&sh.hist[(sh.cand_key[c] >> 8) & 0xFFFu], 1u);
+    __syncthreads();
+    find_digit<THREADS>(sh, 8, kSelBins);
+    const uint32_t prefix1 = sh.prefix;
+    zero_hist<THREADS>(sh, kLastBins);
+    __syncthreads();
     for (uint32_t c = tid; c < n_cand; c += THREADS) {
       const uint32_t kc = sh.cand_key[c];
-      const int pc = sh.cand_pos[c];
-      uint32_t rank = 0, greater = 0;
-      for (uint32_t j = 0; j < n_cand; ++j) {
-        const uint32_t kj = sh.cand_key[j];
-        greater += kj > kc;
-        rank += kj > kc || (kj == kc && sh.cand_pos[j] < pc);
-      }
-      if (rank == rem0 - 1) { sh.kth = kc; sh.need = rem0 - greater; }
+      if ((kc & 0xFFFFFF00u) == prefix1) atomicAdd(&sh.hist[kc & 0xFFu], 1u);
     }
     __syncthreads();
+    find_digit<THREADS>(sh, 0, kLastBins);
   } else {
-    // ---- many keys share the first digit: two more radix passes
-    uint32_t mask = 0xFFF00000u;
-#pragma unroll 1
-    for (int pass = 1; pass < 3; ++pass) {
-      const int shift = pass == 1 ? 8 : 0;
-      const uint32_t dmask = pass == 1 ? 0xFFFu : 0xFFu;
-      for (int b = tid; b < kSelBins; b += THREADS) sh.hist[b] = 0u;
-      __syncthreads();
-      const uint32_t prefix = sh.prefix;
-#pragma unroll
-      for (int e = 0; e < kRegEPT; ++e)
-        if (e < cnt && (key[e] & mask) == prefix) atomicAdd(&sh.hist[(key[e] >> shift) & dmask], 1u);
-      __syncthreads();
-      find_digit<THREADS>(sh, shift, pass == 1 ? kSelBins : 256 < THREADS ? THREADS : 256);
-      mask |= dmask << shift;
-    }
-    if (tid == 0) { sh.kth = sh.prefix; sh.need = sh.remaining; }
+    // many keys share the first digit: the same two passes over the registers
     __syncthreads();
+#pragma unroll
+    for (int e = 0; e < EPT; ++e)
+      if (e < cnt && (key[e] & 0xFFF00000u) == prefix0) atomicAdd(&sh.hist[(key[e] >> 8) & 0xFFFu], 1u);
+    __syncthreads();
+    find_digit<THREADS>(sh, 8, kSelBins);
+    const uint32_t prefix1 = sh.prefix;
+    zero_hist<THREADS>(sh, kLastBins);
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < EPT; ++e)
+      if (e < cnt && (key[e] & 0xFFFFFF00u) == prefix1) atomicAdd(&sh.hist[key[e] & 0xFFu], 1u);
+    __syncthreads();
+    find_digit<THREADS>(sh, 0, kLastBins);
   }
-  const uint32_t kth = sh.kth, need = sh.need;
+  const uint32_t kth = sh.prefix, need = sh.remaining;
   // ---- ordered output
   uint32_t gt = 0, eq = 0;
 #pragma unroll
-  for (int e = 0; e < kRegEPT; ++e)
+  for (int e = 0; e < EPT; ++e)
     if (e < cnt) { gt += key[e] > kth; eq += key[e] == kth; }
   uint32_t total;
   const uint32_t before = block_exclusive_scan<THREADS>((gt << 16) | eq, sh, total);
   uint32_t gt_run = before >> 16, eq_run = before & 0xFFFFu;
 #pragma unroll
-  for (int e = 0; e < kRegEPT; ++e) {
+  for (int e = 0; e < EPT; ++e) {
     if (e >= cnt) break;
     const uint32_t kv = key[e];
     if (kv > kth) {
@@ -192,6 +200,16 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
   }
 }
 
+// Runs select_row_reg with the smallest register block that holds n keys
+// (n <= THREADS * kRegEPT).
+template <int THREADS, typename Map>
+__device__ __forceinline__ void select_row_reg_any(const float* __restrict__ scores, int n, int k, int k_out,
+                                                   int* __restrict__ out, Map map, RegSelSmem<THREADS>& sh) {
+  if (n <= THREADS * 8) select_row_reg<THREADS, 8>(scores, n, k, k_out, out, map, sh);
+  else if (n <= THREADS * 16) select_row_reg<THREADS, 16>(scores, n, k, k_out, out, map, sh);
+  else select_row_reg<THREADS, kRegEPT>(scores, n, k, k_out, out, map, sh);
+}
+
 // Flat rows: row (b, i) keeps the k best of its visible entries.
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS)
@@ -201,7 +219,7 @@ select_flat_reg_kernel(const float* __restrict__ S, const int* __restrict__ q_po
   const int b = blockIdx.y, m = blockIdx.x;
   const size_t row = (size_t)b * T_ + i0 + m;
   const int n = visible_entries(q_pos[row], r, nc);
-  select_row_reg<THREADS>(S + ((size_t)b * nq + m) * ldS, n, k, k, idx + row * k, IdentityMap{}, sh);
+  select_row_reg_any<THREADS>(S + ((size_t)b * nq + m) * ldS, n, k, k, idx + row * k, IdentityMap{}, sh);
 }
 
 // HISA stage 1: the partial block (if any) is always kept; the best full blocks
@@ -219,7 +237,7 @@ select_blocks_reg_kernel(const float* __restrict__ SB, const int* __restrict__ q
   const int k1 = top_m - (partial ? 1 : 0);
   int* out = blk + ((size_t)b * nq + m) * top_m;
   if (k1 > 0) {
-    select_row_reg<THREADS>(SB + ((size_t)b * nq + m) * ldB, full, k1, top_m, out, IdentityMap{}, sh);
+    select_row_reg_any<THREADS>(SB + ((size_t)b * nq + m) * ldB, full, k1, top_m, out, IdentityMap{}, sh);
   } else {
     for (int i = threadIdx.x; i < top_m; i += THREADS) out[i] = -1;
   }
@@ -236,8 +254,8 @@ select_cand_reg_kernel(const float* __restrict__ SC, const int* __restrict__ n_c
   const int b = blockIdx.y, m = blockIdx.x;
   const size_t row = (size_t)b * T_ + i0 + m;
   const size_t slot = (size_t)b * nq + m;
-  select_row_reg<THREADS>(SC + slot * ((size_t)top_m * block), n_cand[slot], k, k, idx + row * k,
-                          BlockListMap{blk + slot * top_m, block}, sh);
+  select_row_reg_any<THREADS>(SC + slot * ((size_t)top_m * block), n_cand[slot], k, k, idx + row * k,
+                              BlockListMap{blk + slot * top_m, block}, sh);
 }
 
 }  // namespace hyb
