@@ -14,7 +14,7 @@
 //               dense range, then the window) into source rows in shared memory
 //               one group ahead, so no role waits on a global index load; also
 //               loads each query's Q tile (2-D TMA, double-buffered);
-//   warps 2-4   K tiles, warps 5-7 V tiles: gathered rows are copied with
+//   warps 2-6   K tiles, warps 7-11 V tiles: gathered rows are copied with
 //               16-byte cp.async by all 96 lanes (the per-SM gather rate grows
 //               with the number of issuing warps), written in the 128-byte
 //               swizzled layout; a window tile whose rows are consecutive is one
@@ -25,8 +25,8 @@
 //               issued before O^T of group g, so the tensor core computes the
 //               next group's scores while the softmax warps turn the current
 //               scores into probabilities;
-//   warps 8-15  softmax and epilogue: thread = key lane (TMEM lane quadrant =
-//               warp % 4), warps 8-11 own heads 0-31 and warps 12-15 heads 32-63.
+//   warps 12-19 softmax and epilogue: thread = key lane (TMEM lane quadrant =
+//               warp % 4), warps 12-15 own heads 0-31 and warps 16-19 heads 32-63.
 // Tensor memory: two S^T buffers (3 tiles x 64 columns) and two O^T
 // accumulators (64 columns), 512 columns in all.
 //
@@ -52,15 +52,26 @@ namespace attn_tc {
 
 constexpr int kH = 64, kD = 128, kTile = 128;
 constexpr int kGT = 3;                                  // tiles per group
-constexpr int kQSt = 2, kKSt = 2, kVSt = 2, kPSt = 2, kTbl = 8;
-constexpr int kThreads = 512;
+// One Q slot (the next query's Q loads while the softmax finishes the current
+// one), three V slots (a V tile may load while the O^T update two tiles back
+// still waits for probabilities), four key-table slots.
+constexpr int kQSt = 1, kKSt = 2, kVSt = 3, kPSt = 2, kTbl = 4;
 constexpr int kProdWarps = 3;                           // per tensor (K, V)
 constexpr int kProdLanes = kProdWarps * 32;
+constexpr int kSmxWarp0 = (2 + 2 * kProdWarps + 3) / 4 * 4;   // first softmax warp (warpgroup-aligned)
+constexpr int kThreads = (kSmxWarp0 + 8) * 32;
+// Register split per warpgroup (setmaxnreg): warps below kSmxWarp0 drop to kRegLow,
+// the 8 softmax warps rise to kRegHigh; the sum stays within the launch allocation
+// (65536 / kThreads rounded down to a multiple of 8, per thread).
+constexpr int kRegLow = 56, kRegHigh = 200;
+static_assert(kRegLow * 32 * kSmxWarp0 + kRegHigh * 256 <= (65536 / kThreads) / 8 * 8 * kThreads,
+              "register split exceeds the launch allocation");
 constexpr int kQBytes = kH * kD * 2;                    // 16 KB, two 64-column sub-tiles
 constexpr int kKVBytes = kTile * kD * 2;                // 32 KB, two 64-column sub-tiles
 constexpr int kPBytes = kTile * kH * 2;                 // 16 KB
-constexpr int kOBytes = kH * kD * 2;                    // 16 KB bf16 output tile, [h][d]
-constexpr int kSmem = kQSt * kQBytes + kKSt * kKVBytes + kVSt * kKVBytes + kPSt * kPBytes + kOBytes + 1024;
+constexpr int kOBytes = kH * kD * 2;                    // 16 KB bf16 output tile [h][d], staged in P slot 0
+static_assert(kOBytes <= kPBytes, "the output tile is staged in a P slot");
+constexpr int kSmem = kQSt * kQBytes + kKSt * kKVBytes + kVSt * kKVBytes + kPSt * kPBytes + 1024;
 constexpr uint32_t kSCols = kGT * kH;                   // 192 columns per S^T buffer
 constexpr uint32_t kOCol = 2 * kSCols;                  // O^T buffers at 384 and 448
 constexpr float kRescaleThreshold = 8.f;                // base-2 units
@@ -202,7 +213,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   uint8_t* sK = sQ + kQSt * kQBytes;
   uint8_t* sV = sK + kKSt * kKVBytes;
   uint8_t* sP = sV + kVSt * kKVBytes;
-  uint8_t* sO = sP + kPSt * kPBytes;
+  uint8_t* sO = sP;   // output staging: P slot 0, idle once the query's last O^T update is done
 
   __shared__ uint64_t q_full[kQSt], q_empty[kQSt], k_full[kKSt], k_empty[kKSt], v_full[kVSt], v_empty[kVSt];
   __shared__ uint64_t s_full[2], s_free[2], p_full[kPSt], p_empty[kPSt], o_full[2], o_ready[2];
@@ -238,10 +249,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   const uint32_t tmem = tmem_base;
   const float c2 = a.scale * 1.4426950408889634f;  // scale * log2(e)
 
-  // Register split per warpgroup.  Launch: 512 threads x 128 = 65536 registers;
-  // after the split 256 x 56 (warps 0-7) + 256 x 200 (warps 8-15) = 65536.
-  if (warp < 8) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+  // Register split per warpgroup (kRegLow / kRegHigh, see their definition).
+  if (warp < kSmxWarp0) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegLow) : "memory");
   if (warp == 1) {
     // ======================================================== key tables and Q
     // Q tiles are queued and issued by lane 0 whenever their slot is free, so
@@ -338,7 +348,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
       }
     }
   } else if (warp >= 2) {
-    // ======================================================== K (warps 2-4) and V (warps 5-7) producers
+    // ======================================================== K and V producers (kProdWarps each)
     const bool is_k = warp < 2 + kProdWarps;
     const int plane = (warp - (is_k ? 2 : 2 + kProdWarps)) * 32 + lane;   // 0 .. kProdLanes-1
     uint32_t G = 0, tiles = 0;
@@ -353,11 +363,12 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         const int slot = G % kTbl;
         ok = mbar_wait(&t_full[slot], full_par(G, kTbl), &abort_flag);
         for (int j = 0; j < nt && ok; ++j, ++tiles) {
-          const int st = tiles % 2;
+          const int nst = is_k ? kKSt : kVSt;
+          const int st = tiles % nst;
           uint64_t* empty = is_k ? &k_empty[st] : &v_empty[st];
           uint64_t* full = is_k ? &k_full[st] : &v_full[st];
           uint8_t* dst = (is_k ? sK : sV) + st * kKVBytes;
-          if (lane == 0) ok = mbar_wait(empty, empty_par(tiles, 2), &abort_flag);
+          if (lane == 0) ok = mbar_wait(empty, empty_par(tiles, nst), &abort_flag);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
           const int first = tbl.first[slot][j];
@@ -535,10 +546,10 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     }
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
-    // ======================================================== softmax + epilogue (warps 8..15)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegHigh) : "memory");
+    // ======================================================== softmax + epilogue (8 warps from kSmxWarp0)
     const int quad = warp & 3;
-    const int hf = (warp - 8) >> 2;                   // head half: heads 32*hf .. 32*hf+31
+    const int hf = (warp - kSmxWarp0) >> 2;           // head half: heads 32*hf .. 32*hf+31
     const int kk = quad * 32 + lane;                  // key lane of a tile; head-dim lane of O^T
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     uint32_t G = 0, n = 0, pt = 0;
@@ -596,6 +607,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         }
         warp_xmax32(mx, lane);
         red[hf][quad][lane] = mx[0] * c2;
+        // P slot 0 held the previous query's output tile: its bulk store must have
+        // read it before this query's probabilities are written there
+        if (first && warp == kSmxWarp0 && lane == 0) bulk_wait_read_all();
         named_sync_softmax();
         if (quad == 0) {
           const int h = hf * 32 + lane;
@@ -687,7 +701,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         fence_after_sync();
         warp_xsum32(lp, lane);
         red[hf][quad][lane] = lp[0];
-        if (warp == 8 && lane == 0) bulk_wait_read_all();   // the previous item's output tile has left sO
+        if (warp == kSmxWarp0 && lane == 0) bulk_wait_read_all();   // the previous item's output tile has left sO
         named_sync_softmax();
         if (quad == 0) {
           const int h = hf * 32 + lane;
@@ -714,7 +728,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           }
           fence_proxy_async_smem();
           named_sync_softmax();
-          if (warp == 8 && lane == 0) {
+          if (warp == kSmxWarp0 && lane == 0) {
             bulk_store_s2g(static_cast<bf16*>(a.o) + prow * kD, smem_u32(sO), kOBytes);
             bulk_commit();
           }
@@ -730,7 +744,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
       }
       ++n;
     }
-    if (warp == 8 && lane == 0) bulk_wait_all();
+    if (warp == kSmxWarp0 && lane == 0) bulk_wait_all();
   }
   fence_before_sync();
   __syncthreads();
