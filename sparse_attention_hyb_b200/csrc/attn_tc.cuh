@@ -380,22 +380,35 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
                 tma_load_2d(dst + c * (kKVBytes / 2), is_k ? &maps.kw : &maps.vw, full, c * 64, first);
             }
           } else {
-            // gathered rows: 16-byte cp.async per lane, lane-consecutive chunks of a
-            // 256-byte row, written with the 128-byte swizzle the MMA descriptors expect;
-            // a masked key's row is zero-filled without reading global memory
+            // gathered rows: a lane owns one 16-byte chunk position of a row in both
+            // 64-column halves; all of its row indices are read from the table first
+            // so that its copies issue back to back (a shared-memory read between
+            // copies halves the gather rate).  Copies are written with the 128-byte
+            // swizzle the MMA descriptors expect; a masked key's row is zero-filled
+            // without reading global memory.
+            constexpr int kTasks = kTile * 8;                       // (row, chunk) pairs per tile
+            constexpr int kIt = (kTasks + kProdLanes - 1) / kProdLanes;
             const int safe = tbl.safe[slot][j];
             const bool win = tbl.win[slot][j] != 0;
             const char* src = static_cast<const char*>(is_k ? (win ? a.kw : a.kc) : (win ? a.vw : a.vc));
             const int* trow = tbl.rows[slot] + j * kTile;
             const uint32_t dbase = smem_u32(dst);
-#pragma unroll 4
-            for (int i = 0; i < (kTile * 16 + kProdLanes - 1) / kProdLanes; ++i) {
+            int rw[kIt];
+#pragma unroll
+            for (int i = 0; i < kIt; ++i) {
               const int q = i * kProdLanes + plane;
-              if (q < kTile * 16) {
-                const int r = q >> 4, c = (q >> 3) & 1, ch = q & 7;
-                const int rw = trow[r];
-                cp_async16_zfill(dbase + c * (kKVBytes / 2) + r * 128 + ((ch ^ (r & 7)) << 4),
-                                 src + (size_t)(rw >= 0 ? rw : safe) * (kD * 2) + c * 128 + ch * 16, rw >= 0 ? 16u : 0u);
+              rw[i] = q < kTasks ? trow[q >> 3] : -1;
+            }
+#pragma unroll
+            for (int i = 0; i < kIt; ++i) {
+              const int q = i * kProdLanes + plane;
+              if (q < kTasks) {
+                const int r = q >> 3, ch = q & 7;
+                const char* row = src + (size_t)(rw[i] >= 0 ? rw[i] : safe) * (kD * 2) + ch * 16;
+                const uint32_t d = dbase + r * 128 + ((ch ^ (r & 7)) << 4);
+                const uint32_t nb = rw[i] >= 0 ? 16u : 0u;
+                cp_async16_zfill(d, row, nb);
+                cp_async16_zfill(d + kKVBytes / 2, row + 128, nb);
               }
             }
           }
@@ -444,8 +457,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         }
         if (s_have && pc < kRing) {
           const int sb = Gs % 2, qb = ns % kQSt;
-          if (!s_open && mbar_try_wait(&s_free[sb], empty_par(Gs, 2)) &&
-              (!s_first || mbar_try_wait(&q_full[qb], full_par(ns, kQSt)))) {
+          if (!s_open && mbar_test_wait(&s_free[sb], empty_par(Gs, 2)) &&
+              (!s_first || mbar_test_wait(&q_full[qb], full_par(ns, kQSt)))) {
             s_open = true;
             s_nt = min(kGT, s_it.tile_end - s_g0);
             s_j = 0;
@@ -453,7 +466,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           if (s_open) {
             while (s_j < s_nt) {
               const int ks = kt % kKSt;
-              if (!mbar_try_wait(&k_full[ks], full_par(kt, kKSt))) break;
+              if (!mbar_test_wait(&k_full[ks], full_par(kt, kKSt))) break;
               fence_after_sync();
               fence_async_shared();
               const uint32_t d = tmem + sb * kSCols + s_j * kH;
@@ -491,7 +504,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         }
         if (pc > 0) {
           const PendingPV pv = ring[ph];
-          if (!p_open && mbar_try_wait(&o_ready[pv.ob], full_par(ordy[pv.ob], 1))) {
+          if (!p_open && mbar_test_wait(&o_ready[pv.ob], full_par(ordy[pv.ob], 1))) {
             ++ordy[pv.ob];
             p_open = true;
             p_j = 0;
@@ -500,7 +513,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           if (p_open) {
             while (p_j < pv.ntiles) {
               const int vs = vt % kVSt, ps = pt % kPSt;
-              if (!mbar_try_wait(&v_full[vs], full_par(vt, kVSt)) || !mbar_try_wait(&p_full[ps], full_par(pt, kPSt))) break;
+              if (!mbar_test_wait(&v_full[vs], full_par(vt, kVSt)) || !mbar_test_wait(&p_full[ps], full_par(pt, kPSt))) break;
               fence_after_sync();
               fence_async_shared();
               const uint32_t vbase = smem_u32(sV + vs * kKVBytes);
