@@ -293,6 +293,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
       if (lane == 0) {   // (q_next is lane 0's; the queue cannot fill while the table ring holds fewer groups)
         if (n - q_next >= kQQ && wait_serving(&q_empty[q_next % kQSt], empty_par(q_next, kQSt))) service_q();
         qrow[n % kQQ] = it.kl.row;
+        for (int c = 0; c < 2; ++c) tma_prefetch_2d(&maps.q, c * 64, it.kl.row * kH);   // into L2, ahead of its slot
       }
       ++n;
       service_q();

@@ -11,7 +11,9 @@
 //               (M=128, N=256, K=16 steps) into one of two 256-column
 //               accumulators and commits them to the ring / epilogue barriers;
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time from their lane
-//               quadrant and store the fp32 scores (visible columns only).
+//               quadrant, stage each 32 x 32 fp32 block in shared memory
+//               (128-byte swizzle, two buffers per warp) and write it with a
+//               TMA tensor store, so the scores leave as whole lines.
 // Column tiles no row of the CTA can see are never loaded (causal skipping).
 #pragma once
 #include "common.cuh"
@@ -28,13 +30,14 @@ template <int KB>  // dI = 64 * KB
 struct TcScoreSmem {
   static constexpr int kA = KB * kTcBM * 128;          // bytes of the query tile
   static constexpr int kB = KB * kTcBN * 128;          // bytes of one key tile
-  static constexpr int kTotal = kA + kTcStages * kB + 1024;  // + alignment slack
+  static constexpr int kC = 4 * 2 * 32 * 128;         // epilogue staging: 4 warps x 2 buffers x 32 rows x 128 B
+  static constexpr int kTotal = kA + kTcStages * kB + kC + 1024;  // + alignment slack
 };
 
 template <int KB>
 __global__ void __launch_bounds__(kTcThreads, 1)
 scores_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                 const int* __restrict__ q_pos, float* __restrict__ S, int T_, int i0, int nq, int keys_cap,
+                 const __grid_constant__ CUtensorMap map_s, const int* __restrict__ q_pos, int T_, int i0, int nq, int keys_cap,
                  int r, int nc, int div, int ldS, int nsplit) {
   using namespace sm100;
   using L = TcScoreSmem<KB>;
@@ -42,6 +45,7 @@ scores_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + L::kA;
+  uint8_t* sC = sB + kTcStages * L::kB;
   __shared__ uint64_t bar_a, bar_full[kTcStages], bar_empty[kTcStages], bar_tfull[2], bar_tempty[2], bar_done;
   __shared__ uint32_t tmem_base;
   __shared__ int tile_cols;
@@ -135,8 +139,8 @@ scores_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     } else if (warp >= 2) {
       // ---------------- epilogue
       const int quad = warp & 3;
-      const int m = m0 + quad * 32 + lane;
-      float* srow = S + ((size_t)b * nq + m) * ldS;
+      uint8_t* stg = sC + quad * (2 * 32 * 128);
+      uint32_t nst = 0;   // blocks this warp has stored
       for (int it = 0; it < my_tiles; ++it) {
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
@@ -149,24 +153,27 @@ scores_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kTcBN + c * 32, v);
           tmem_wait_ld();
           const int cb = col0 + c * 32;
-          if (m < nq && cb < cols) {
-            if (cb + 32 <= cols) {
-              float4* dst = reinterpret_cast<float4*>(srow + cb);
+          if (cb >= cols) continue;   // columns no row of the CTA can see
+          uint8_t* buf = stg + (nst & 1) * (32 * 128);
+          if (nst >= 2 && lane == 0) bulk_wait_read<1>();   // the store two blocks back has read this buffer
+          __syncwarp();
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                     __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (cb + e < cols) srow[cb + e] = __uint_as_float(v[e]);
-            }
+          for (int e = 0; e < 8; ++e)
+            *reinterpret_cast<uint4*>(buf + lane * 128 + ((e ^ (lane & 7)) << 4)) =
+                make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&map_s, smem_u32(buf), cb, m0 + quad * 32, b);   // rows past nq are clipped
+            bulk_commit();
           }
+          ++nst;
         }
         fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_tempty[acc]);
       }
+      if (lane == 0) bulk_wait_all();
     }
   }
   fence_before_sync();
@@ -187,10 +194,11 @@ inline bool tc_scores_supported(int dI, const void* qi, const void* keys) {
 inline cudaError_t launch_scores_tc(const void* qi, const int* q_pos, const void* keys, float* S, int batch, int T_,
                                     int i0, int nq, int dI, int keys_cap, int r, int nc, int div, int ldS,
                                     int max_cols, cudaStream_t stream) {
-  CUtensorMap mq, mk;
+  CUtensorMap mq, mk, ms;
   if (!make_map_bf16_2d(&mq, qi, (uint64_t)batch * T_, dI, (uint64_t)dI * 2, kTcBM, 64)) return cudaErrorInvalidValue;
   if (!make_map_bf16_2d(&mk, keys, (uint64_t)batch * keys_cap, dI, (uint64_t)dI * 2, kTcBN, 64))
     return cudaErrorInvalidValue;
+  if (!make_map_f32_3d(&ms, S, (uint64_t)ldS, (uint64_t)ldS, (uint64_t)nq, (uint64_t)batch, 32)) return cudaErrorInvalidValue;
   const int m_tiles = (nq + kTcBM - 1) / kTcBM;
   const int n_tiles = (max_cols + kTcBN - 1) / kTcBN;
   int nsplit = (2 * 148 + m_tiles * batch - 1) / (m_tiles * batch);
@@ -202,13 +210,13 @@ inline cudaError_t launch_scores_tc(const void* qi, const int* q_pos, const void
     const int smem = TcScoreSmem<2>::kTotal;
     if ((e = cudaFuncSetAttribute(scores_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
       return e;
-    scores_tc_kernel<2><<<grid, kTcThreads, smem, stream>>>(mq, mk, q_pos, S, T_, i0, nq, keys_cap, r, nc, div,
+    scores_tc_kernel<2><<<grid, kTcThreads, smem, stream>>>(mq, mk, ms, q_pos, T_, i0, nq, keys_cap, r, nc, div,
                                                              ldS, nsplit);
   } else {
     const int smem = TcScoreSmem<1>::kTotal;
     if ((e = cudaFuncSetAttribute(scores_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
       return e;
-    scores_tc_kernel<1><<<grid, kTcThreads, smem, stream>>>(mq, mk, q_pos, S, T_, i0, nq, keys_cap, r, nc, div,
+    scores_tc_kernel<1><<<grid, kTcThreads, smem, stream>>>(mq, mk, ms, q_pos, T_, i0, nq, keys_cap, r, nc, div,
                                                              ldS, nsplit);
   }
   count_launch();

@@ -20,16 +20,19 @@ namespace hyb {
 
 constexpr int kRegEPT = 32;
 constexpr int kSelBins = 4096;       // 12-bit digits
-constexpr int kSelCand = 512;        // boundary-bin candidates resolved by ranking
+constexpr int kSelCand = 512;        // boundary-bin candidates resolved over shared memory
+constexpr int kSelOut = 2048;        // outputs staged in shared memory for coalesced stores (k <= kSelOut)
 
 template <int THREADS>
 struct RegSelSmem {
   alignas(16) uint32_t hist[kSelBins];
   uint32_t cand_key[kSelCand];
+  int outbuf[kSelOut];
   uint32_t warp_tot[THREADS / 32];
   uint32_t warp_off[THREADS / 32];
   uint32_t total;
   uint32_t prefix, remaining, kth, need;
+  uint32_t bin_count, n_slots;   // population of the last found bin; candidate slot counter
 };
 
 // Exclusive prefix sum over the CTA of one value per thread; `total` receives the sum.
@@ -88,6 +91,7 @@ __device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift, i
       if (above + h >= rem) {
         sh.prefix = prefix | ((uint32_t)(threadIdx.x * bpt + e) << shift);
         sh.remaining = rem - above;
+        sh.bin_count = h;
         break;
       }
       above += h;
@@ -127,7 +131,7 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
   constexpr int kLastBins = 256 < THREADS ? THREADS : 256;   // 8-bit pass, at least one bin per thread
   // ---- pass 0: bits 31..20
   zero_hist<THREADS>(sh, kSelBins);
-  if (tid == 0) { sh.prefix = 0; sh.remaining = (uint32_t)k; }
+  if (tid == 0) { sh.prefix = 0; sh.remaining = (uint32_t)k; sh.n_slots = 0; }
   __syncthreads();
 #pragma unroll
   for (int e = 0; e < EPT; ++e)
@@ -135,18 +139,15 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
   __syncthreads();
   find_digit<THREADS>(sh, 20, kSelBins);
   const uint32_t prefix0 = sh.prefix;
-  // ---- the boundary bin's keys
-  uint32_t mine = 0;
-#pragma unroll
-  for (int e = 0; e < EPT; ++e) mine += (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) ? 1u : 0u;
-  uint32_t n_cand;
-  uint32_t slot = block_exclusive_scan<THREADS>(mine, sh, n_cand);
+  // ---- the boundary bin's keys (their number is the bin's count)
+  const uint32_t n_cand = sh.bin_count;
+  __syncthreads();   // every thread has read the histogram results before it is cleared
   zero_hist<THREADS>(sh, kSelBins);
   if (n_cand <= (uint32_t)kSelCand) {
-    // few: compact them and resolve the low 20 bits over the candidates alone
+    // few: gather them (in any order) and resolve the low 20 bits over them alone
 #pragma unroll
     for (int e = 0; e < EPT; ++e)
-      if (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) sh.cand_key[slot++] = key[e];
+      if (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) sh.cand_key[atomicAdd(&sh.n_slots, 1u)] = key[e];
     __syncthreads();
     for (uint32_t c = tid; c < n_cand; c += THREADS) atomicAdd(&sh.hist[(sh.cand_key[c] >> 8) & 0xFFFu], 1u);
     __syncthreads();
@@ -186,17 +187,25 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
   uint32_t total;
   const uint32_t before = block_exclusive_scan<THREADS>((gt << 16) | eq, sh, total);
   uint32_t gt_run = before >> 16, eq_run = before & 0xFFFFu;
+  // selected positions in ascending order: staged in shared memory when k fits,
+  // then stored by consecutive threads
+  const bool staged = k <= kSelOut;
+  int* dst = staged ? sh.outbuf : out;
 #pragma unroll
   for (int e = 0; e < EPT; ++e) {
     if (e >= cnt) break;
     const uint32_t kv = key[e];
     if (kv > kth) {
-      out[gt_run + (eq_run < need ? eq_run : need)] = map(base + e);
+      dst[gt_run + (eq_run < need ? eq_run : need)] = map(base + e);
       ++gt_run;
     } else if (kv == kth) {
-      if (eq_run < need) out[gt_run + eq_run] = map(base + e);
+      if (eq_run < need) dst[gt_run + eq_run] = map(base + e);
       ++eq_run;
     }
+  }
+  if (staged) {
+    __syncthreads();
+    for (int i = tid; i < k; i += THREADS) out[i] = sh.outbuf[i];
   }
 }
 
