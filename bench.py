@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU oracle sample")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the HCA prefill, 128K indexer and 1M-context measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-only", action="store_true", help="time only the prefill step (profiling runs)")
     ap.add_argument("--L", type=int, default=None, help="override the prefill length (profiling runs)")
@@ -356,6 +358,210 @@ def bench_decode(S, steps, warmup, flush):
             "algorithmic_bytes_csa": bytes_csa, "algorithmic_bytes_hca": bytes_hca}
 
 
+# --------------------------------------------------------------------------- the other configs
+
+
+def _rec(ev, i):
+    if ev:
+        ev[i].record()
+
+
+def graph_times(step, n_seg, steps, warmup, flush):
+    """Median time (ms) of each of the n_seg segments of step(ev), replayed as one
+    CUDA graph per step with L2 flushed between replays (outside the events)."""
+    for _ in range(warmup):
+        step(None)
+    torch.cuda.synchronize()
+    graph, ev = capture(step, n_seg + 1)
+    seg = []
+    for _ in range(steps):
+        flush.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        seg.append([ev[j].elapsed_time(ev[j + 1]) for j in range(n_seg)])
+    del graph
+    return [float(x) for x in np.median(np.array(seg), axis=0)]
+
+
+def _dense_flops(w, r, n_c, q_pos):
+    t = q_pos.astype(np.int64)
+    return 4.0 * w.H * w.D * float((np.minimum((t + 1) // r, n_c) + np.minimum(w.W, t + 1)).sum())
+
+
+def bench_hca_prefill(S, st, csa_step_ms, steps, warmup, flush, pk):
+    """HCA layer (r=128, dense over all visible entries + window) on the 32K prefill
+    inputs, and the CSA+HCA pair."""
+    w, raw, qs, A = st.w, st.raw, st.qs, S.abi
+    ly = C.HCA128
+    n_c = w.L // ly.r
+    bias = make.make_bias(w, ly, "cuda")
+    kc = torch.empty(1, n_c, w.D, dtype=raw["xk"].dtype, device="cuda")
+    vc = torch.empty_like(kc)
+    o = torch.empty_like(qs["q"])
+    lse = torch.empty(1, w.T, w.H, dtype=torch.float32, device="cuda")
+
+    def step(ev):
+        _rec(ev, 0)
+        A.hyb_compress(raw["xk"], raw["xv"], None, raw["z"], bias, ly.r, ly.overlap, 0, n_c, kc, vc, None)
+        _rec(ev, 1)
+        A.hyb_attn_fwd(qs["q"], qs["q_pos"], kc, vc, n_c, ly.r, None, 0, raw["xk"], raw["xv"], w.W, st.scale,
+                       o, lse, A.HYB_ATTN_PREFILL, None)
+        _rec(ev, 2)
+
+    comp_ms, attn_ms = graph_times(step, 2, steps, warmup, flush)
+    fl = _dense_flops(w, ly.r, n_c, qs["q_pos"][0].cpu().numpy())
+    ms = comp_ms + attn_ms
+    return {"workload": "hca_prefill_32k_bf16", "tokens_per_s": w.T / (ms / 1e3), "ms": ms,
+            "stages_ms": {"compress": comp_ms, "attention": attn_ms},
+            "attention_tflops": fl / (attn_ms / 1e3) / 1e12,
+            "attention_frac_of_bf16_peak": fl / (attn_ms / 1e3) / 1e12 / pk["bf16_tflops"],
+            "csa_plus_hca_tokens_per_s": w.T / ((csa_step_ms + ms) / 1e3)}
+
+
+def bench_index_128k(S, steps, warmup, flush):
+    """Indexer latency of the last query chunk of a 128K prefill (queries
+    130048..131071, chunk 1024): flat top-2048 over all visible entries vs HISA
+    (128-entry blocks, top-64 blocks, then top-2048 of their entries)."""
+    w = C.PREFILL_128K
+    ly = w.layer("csa")
+    wq = C.scaled(w, T=ly.q_chunk, q_pos0=w.L - ly.q_chunk)
+    A = S.abi
+    n_c = w.L // ly.r
+    raw = make.make_raw(w, "cuda")
+    bias = make.make_bias(w, ly, "cuda")
+    kc, vc, ic = S.layer.compress(raw["xk"], raw["xv"], raw["xi"], raw["z"], bias, ly.r, ly.overlap, n_c)
+    del raw, kc, vc
+    reps = S.layer.block_reps(ic, n_c, ly.block)
+    qs = make.make_queries(wq, "cuda")
+    idx = torch.empty(1, wq.T, ly.k, dtype=torch.int32, device="cuda")
+    idx2 = torch.empty_like(idx)
+    wsf = torch.empty(max(256, A.hyb_index_topk_workspace_size(1, 1, wq.T, n_c, w.dI, ly.k, A.HYB_INDEX_FLAT, 0, 0,
+                                                               0)), dtype=torch.uint8, device="cuda")
+    wsh = torch.empty(max(256, A.hyb_index_topk_workspace_size(1, 1, wq.T, n_c, w.dI, ly.k, A.HYB_INDEX_HISA,
+                                                               ly.block, ly.top_m, ly.q_chunk)),
+                      dtype=torch.uint8, device="cuda")
+
+    def step(ev):
+        _rec(ev, 0)
+        A.hyb_index_topk(qs["qi"], qs["q_pos"], ic, n_c, ly.r, ly.k, A.HYB_INDEX_FLAT, None, 0, 0, 0, idx, wsf)
+        _rec(ev, 1)
+        A.hyb_index_topk(qs["qi"], qs["q_pos"], ic, n_c, ly.r, ly.k, A.HYB_INDEX_HISA, reps, ly.block, ly.top_m,
+                         ly.q_chunk, idx2, wsh)
+        _rec(ev, 2)
+
+    flat_ms, hisa_ms = graph_times(step, 2, steps, warmup, flush)
+    return {"workload": "csa_index_128k_last_chunk_bf16", "queries": wq.T, "k": ly.k,
+            "flat_ms": flat_ms, "hisa_ms": hisa_ms, "hisa_speedup": flat_ms / hisa_ms}
+
+
+def bench_1m(S, steps, warmup, flush, pk):
+    """1M-token context: S1 over the whole prefix (CSA with indexer keys, HCA, HISA
+    block representatives), a batch-1 decode step (CSA with the HISA indexer, HCA)
+    and an 8K-query chunked prefill at the end of the context."""
+    wd, wc = C.CTX_1M_DECODE, C.CTX_1M_CHUNK
+    csa, hca = wd.layer("csa"), wd.layer("hca")
+    A = S.abi
+    L, dt = wd.L, torch.bfloat16
+    raw = make.make_raw(wd, "cuda")                       # L + 1 tokens (the decode token last)
+    ring = make.ring_from_raw(wd, raw)
+    xk, xv, xi, z = (raw[n][:, :L] for n in ("xk", "xv", "xi", "z"))
+    ncc, nch = L // csa.r, L // hca.r
+    bias_c, bias_h = make.make_bias(wd, csa, "cuda"), make.make_bias(wd, hca, "cuda")
+    kc_c = torch.empty(1, ncc, wd.D, dtype=dt, device="cuda")
+    vc_c, ic_c = torch.empty_like(kc_c), torch.empty(1, ncc, wd.dI, dtype=dt, device="cuda")
+    kc_h = torch.empty(1, nch, wd.D, dtype=dt, device="cuda")
+    vc_h = torch.empty_like(kc_h)
+    nb = ncc // csa.block
+    reps = torch.empty(1, nb, wd.dI, dtype=dt, device="cuda")
+
+    def s1(ev):
+        _rec(ev, 0)
+        A.hyb_compress(xk, xv, xi, z, bias_c, csa.r, csa.overlap, 0, ncc, kc_c, vc_c, ic_c)
+        A.hyb_block_reps(ic_c, csa.block, 0, nb, reps)
+        _rec(ev, 1)
+        A.hyb_compress(xk, xv, None, z, bias_h, hca.r, hca.overlap, 0, nch, kc_h, vc_h, None)
+        _rec(ev, 2)
+
+    s1_csa_ms, s1_hca_ms = graph_times(s1, 2, steps, warmup, flush)
+    s1_bytes_csa = L * (2 * wd.D + wd.dI) * 2 + L * 4 + ncc * (2 * wd.D + wd.dI) * 2 + nb * wd.dI * 2
+    s1_bytes_hca = L * 2 * wd.D * 2 + L * 4 + nch * 2 * wd.D * 2
+    scale = 1.0 / math.sqrt(wd.D)
+    # ---- decode step, batch 1
+    qd = make.make_queries(wd, "cuda")
+    idx_d = torch.empty(1, 1, csa.k, dtype=torch.int32, device="cuda")
+    od, od2 = torch.empty_like(qd["q"]), torch.empty_like(qd["q"])
+    lsed = torch.empty(1, 1, wd.H, dtype=torch.float32, device="cuda")
+    lsed2 = torch.empty_like(lsed)
+    wsi = torch.empty(max(256, A.hyb_index_topk_workspace_size(1, 1, 1, ncc, wd.dI, csa.k, A.HYB_INDEX_HISA,
+                                                               csa.block, csa.top_m, 0)), dtype=torch.uint8,
+                      device="cuda")
+    wsa = torch.empty(max(256, A.hyb_attn_fwd_workspace_size(1, 1, 1, wd.H, wd.D, csa.k, ncc, wd.W, 1)),
+                      dtype=torch.uint8, device="cuda")
+    wsh = torch.empty(max(256, A.hyb_attn_fwd_workspace_size(1, 1, 1, wd.H, wd.D, 0, nch, wd.W, 1)),
+                      dtype=torch.uint8, device="cuda")
+
+    def dec(ev):
+        _rec(ev, 0)
+        A.hyb_index_topk(qd["qi"], qd["q_pos"], ic_c, ncc, csa.r, csa.k, A.HYB_INDEX_HISA, reps, csa.block,
+                         csa.top_m, 0, idx_d, wsi)
+        A.hyb_attn_fwd(qd["q"], qd["q_pos"], kc_c, vc_c, ncc, csa.r, idx_d, csa.k, ring["kw"], ring["vw"], wd.W,
+                       scale, od, lsed, A.HYB_ATTN_DECODE, wsa)
+        _rec(ev, 1)
+        A.hyb_attn_fwd(qd["q"], qd["q_pos"], kc_h, vc_h, nch, hca.r, None, 0, ring["kw"], ring["vw"], wd.W, scale,
+                       od2, lsed2, A.HYB_ATTN_DECODE, wsh)
+        _rec(ev, 2)
+
+    dec_csa_ms, dec_hca_ms = graph_times(dec, 2, steps, warmup, flush)
+    cand = csa.top_m * csa.block
+    dec_bytes_csa = nb * wd.dI * 2 + cand * wd.dI * 2 + (csa.k + wd.W) * 2 * wd.D * 2 + 2 * wd.H * wd.D * 2
+    dec_bytes_hca = (nch + wd.W) * 2 * wd.D * 2 + 2 * wd.H * wd.D * 2
+    # ---- 8K-query chunked prefill at the end of the context
+    qc = make.make_queries(wc, "cuda")
+    idx_c = torch.empty(1, wc.T, csa.k, dtype=torch.int32, device="cuda")
+    oc, oc2 = torch.empty_like(qc["q"]), torch.empty_like(qc["q"])
+    lsec = torch.empty(1, wc.T, wd.H, dtype=torch.float32, device="cuda")
+    lsec2 = torch.empty_like(lsec)
+    wsc = torch.empty(max(256, A.hyb_index_topk_workspace_size(1, 1, wc.T, ncc, wd.dI, csa.k, A.HYB_INDEX_HISA,
+                                                               csa.block, csa.top_m, 1024)), dtype=torch.uint8,
+                      device="cuda")
+
+    def chunk(ev):
+        _rec(ev, 0)
+        A.hyb_index_topk(qc["qi"], qc["q_pos"], ic_c, ncc, csa.r, csa.k, A.HYB_INDEX_HISA, reps, csa.block,
+                         csa.top_m, 1024, idx_c, wsc)
+        _rec(ev, 1)
+        A.hyb_attn_fwd(qc["q"], qc["q_pos"], kc_c, vc_c, ncc, csa.r, idx_c, csa.k, xk, xv, wd.W, scale, oc, lsec,
+                       A.HYB_ATTN_PREFILL, None)
+        _rec(ev, 2)
+        A.hyb_attn_fwd(qc["q"], qc["q_pos"], kc_h, vc_h, nch, hca.r, None, 0, xk, xv, wd.W, scale, oc2, lsec2,
+                       A.HYB_ATTN_PREFILL, None)
+        _rec(ev, 3)
+
+    idx_ms, attn_c_ms, attn_h_ms = graph_times(chunk, 3, steps, warmup, flush)
+    qp = qc["q_pos"][0].cpu().numpy().astype(np.int64)
+    fl_c = 4.0 * wd.H * wd.D * float((np.minimum(np.minimum((qp + 1) // csa.r, ncc), csa.k)
+                                       + np.minimum(wd.W, qp + 1)).sum())
+    fl_h = _dense_flops(wc, hca.r, nch, qp)
+    hbm = pk["hbm_gbs"]
+    return {
+        "s1_1m": {"csa_ms": s1_csa_ms, "hca_ms": s1_hca_ms,
+                  "csa_hbm_gbs": s1_bytes_csa / (s1_csa_ms / 1e3) / 1e9,
+                  "hca_hbm_gbs": s1_bytes_hca / (s1_hca_ms / 1e3) / 1e9,
+                  "csa_frac_of_hbm": s1_bytes_csa / (s1_csa_ms / 1e3) / 1e9 / hbm,
+                  "hca_frac_of_hbm": s1_bytes_hca / (s1_hca_ms / 1e3) / 1e9 / hbm},
+        "decode_bs1_ctx1m": {"csa_hisa_ms": dec_csa_ms, "hca_ms": dec_hca_ms,
+                             "tokens_per_s_csa_plus_hca": 1.0 / ((dec_csa_ms + dec_hca_ms) / 1e3),
+                             "csa_hbm_gbs": dec_bytes_csa / (dec_csa_ms / 1e3) / 1e9,
+                             "hca_hbm_gbs": dec_bytes_hca / (dec_hca_ms / 1e3) / 1e9},
+        "chunk_prefill_8k_at_1m": {"csa_index_hisa_ms": idx_ms, "csa_attention_ms": attn_c_ms,
+                                   "hca_attention_ms": attn_h_ms,
+                                   "tokens_per_s_csa": wc.T / ((idx_ms + attn_c_ms) / 1e3),
+                                   "tokens_per_s_hca": wc.T / (attn_h_ms / 1e3),
+                                   "csa_attention_tflops": fl_c / (attn_c_ms / 1e3) / 1e12,
+                                   "hca_attention_tflops": fl_h / (attn_h_ms / 1e3) / 1e12},
+    }
+
+
 # --------------------------------------------------------------------------- CPU oracle
 
 
@@ -436,12 +642,21 @@ def run_ours(args, world, rank, local):
     peak = pk["bf16_tflops"]
     traffic = measured_traffic("attention")
     if args.prefill_only:
-        args.no_decode = args.no_cpu_baseline = True
+        args.no_decode = args.no_cpu_baseline = args.no_extras = True
         e2e_ms, h2d, d2h = float("nan"), 0, 0
     else:
         e2e_ms, h2d, d2h = bench_e2e(S, st, max(3, args.steps // 2))
         e2e_ms = max_over_ranks(e2e_ms, world)
     decode = None if args.no_decode else bench_decode(S, args.steps, args.warmup, flush)
+    extras = None
+    if not args.no_extras:
+        extras = {"hca_prefill_32k": bench_hca_prefill(S, st, step_ms, args.steps, args.warmup, flush, pk)}
+        del st
+        torch.cuda.empty_cache()
+        extras["index_128k_last_chunk"] = bench_index_128k(S, args.steps, args.warmup, flush)
+        torch.cuda.empty_cache()
+        extras.update(bench_1m(S, args.steps, args.warmup, flush, pk))
+        extras["timing"] = "median of the timed steps, CUDA-graph replay, L2 flushed between steps"
     if S.abi.hyb_get_device_status() != 0:
         raise RuntimeError("device status error after the benchmark")
     cpu = None
@@ -470,6 +685,7 @@ def run_ours(args, world, rank, local):
                 "d2h_bytes_per_step": d2h},
         "clocks": clocks,
         "decode": decode,
+        "extras": extras,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)

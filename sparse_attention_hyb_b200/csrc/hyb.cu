@@ -10,6 +10,7 @@
 #include "topk.cuh"
 #include "index.cuh"
 #include "index_tc.cuh"
+#include "hisa_tc.cuh"
 #include "topk_reg.cuh"
 #include "attn.cuh"
 #include "attn_tc.cuh"
@@ -44,7 +45,8 @@ struct IndexPlan {
   int nq;        // queries per chunk (per batch)
   int ldS;       // flat: score row stride; HISA: block-score row stride
   int nb;        // HISA: blocks with a representative
-  size_t off_scores, off_blk, off_ncand, off_cand, off_keys, total;
+  size_t off_scores, off_blk, off_ncand, off_cand, off_keys, off_list, off_work, off_nwork, total;
+  int work_cap;  // HISA grouped stage 2: work items per batch
   bool global_keys;
 };
 
@@ -70,6 +72,10 @@ IndexPlan plan_index(int dtype, int batch, int T, int nc, int k, int mode, int b
     p.off_blk = off;    off += align_up((size_t)batch * p.nq * top_m * 4);
     p.off_ncand = off;  off += align_up((size_t)batch * p.nq * 4);
     p.off_cand = off;   off += align_up((size_t)batch * p.nq * cand * 4);
+    p.work_cap = hisa_work_cap(p.nq, top_m, p.nb + 1);
+    p.off_list = off;   off += align_up((size_t)batch * p.nq * top_m * 4);
+    p.off_work = off;   off += align_up((size_t)batch * p.work_cap * sizeof(HgWork));
+    p.off_nwork = off;  off += align_up((size_t)batch * 4);
     p.total = off;
   }
   return p;
@@ -126,12 +132,10 @@ int index_topk_impl(int batch, int T_, int dI, const void* qi, const int* q_pos,
       int* blk = reinterpret_cast<int*>(ws + p.off_blk);
       int* ncand = reinterpret_cast<int*>(ws + p.off_ncand);
       float* SC = reinterpret_cast<float*>(ws + p.off_cand);
-      if (p.nb > 0) {
-        dim3 g((p.nb + kSB_N - 1) / kSB_N, (nq + kSB_M - 1) / kSB_M, batch);
-        scores_ffma_kernel<T><<<g, 256, 0, stream>>>((const T*)qi, q_pos, (const T*)reps, S, T_, i0, nq,
-                                                     dI, nb_cap, r, nc, block, p.ldS);
-      count_launch();
-      }
+      if (p.nb > 0 &&
+          (e = launch_scores<T>(qi, q_pos, reps, S, batch, T_, i0, nq, dI, nb_cap, r, nc, block, p.ldS, stream)) !=
+              cudaSuccess)
+        return HYB_ERR_CUDA;
       if (p.nb <= 256 * kRegEPT) {
         select_blocks_reg_kernel<256><<<dim3(nq, batch), 256, 0, stream>>>(S, q_pos, blk, T_, i0, nq, r, nc, block,
                                                                           top_m, p.ldS);
@@ -145,9 +149,21 @@ int index_topk_impl(int batch, int T_, int dI, const void* qi, const int* q_pos,
                                                                                nc, block, top_m, p.ldS);
       }
       count_launch();
-      hisa_cand_scores_kernel<T><<<dim3(nq, batch), 256, dI * 4, stream>>>(
-          (const T*)qi, q_pos, (const T*)ic, blk, SC, ncand, T_, i0, nq, dI, nc_cap, r, nc, block, top_m);
-      count_launch();
+      if (hisa_grouped_supported<T>(dI, block, p.nb, qi, ic)) {
+        int* list = reinterpret_cast<int*>(ws + p.off_list);
+        HgWork* work = reinterpret_cast<HgWork*>(ws + p.off_work);
+        int* nwork = reinterpret_cast<int*>(ws + p.off_nwork);
+        hisa_group_kernel<<<batch, kHgThreads, 0, stream>>>(q_pos, blk, ncand, list, work, nwork, T_, i0, nq, r, nc,
+                                                            block, top_m, p.nb + 1, p.work_cap);
+        count_launch();
+        if ((e = launch_hisa_block_mma(qi, ic, list, work, nwork, SC, batch, T_, i0, nq, dI, nc_cap, top_m,
+                                       p.work_cap, stream)) != cudaSuccess)
+          return HYB_ERR_CUDA;
+      } else {
+        hisa_cand_scores_kernel<T><<<dim3(nq, batch), 256, dI * 4, stream>>>(
+            (const T*)qi, q_pos, (const T*)ic, blk, SC, ncand, T_, i0, nq, dI, nc_cap, r, nc, block, top_m);
+        count_launch();
+      }
       const int n2 = top_m * block;
       if (n2 <= 256 * kRegEPT) {
         select_cand_reg_kernel<256><<<dim3(nq, batch), 256, 0, stream>>>(SC, ncand, blk, idx, T_, i0, nq, block,
