@@ -80,6 +80,7 @@ constexpr int kTblArrivals = 2 * kProdLanes + 256;      // K producers, V produc
 struct Maps {
   CUtensorMap q;        // [batch*T*H, D], 64 x 64 boxes
   CUtensorMap kw, vw;   // [batch*ring, D], 128-row x 64-column boxes (contiguous window tiles)
+  CUtensorMap kc, vc;   // [batch*nc_cap, D], same boxes (full tiles of a dense compressed range)
 };
 
 // Per-query key list: compressed slots [0, n_comp) padded to whole tiles, then
@@ -331,6 +332,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
             if (win) {   // window positions are consecutive rows unless the ring wraps inside the tile
               const int s0 = (it.kl.w0 + (g0 + j - it.kl.comp_tiles) * kTile) % a.ring;
               if (s0 + kTile <= a.ring) first = base + s0;
+            } else if (!a.idx && (g0 + j + 1) * kTile <= it.kl.n_comp) {
+              first = base + (g0 + j) * kTile;   // a full tile of the dense compressed range
             }
             tbl.first[slot][j] = first;
           }
@@ -354,7 +357,10 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     const int plane = (warp - (is_k ? 2 : 2 + kProdWarps)) * 32 + lane;   // 0 .. kProdLanes-1
     uint32_t G = 0, tiles = 0;
     bool ok = true;
-    if (plane == 0) prefetch_tmap(is_k ? &maps.kw : &maps.vw);
+    if (plane == 0) {
+      prefetch_tmap(is_k ? &maps.kw : &maps.vw);
+      prefetch_tmap(is_k ? &maps.kc : &maps.vc);
+    }
     for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
       Item it;
       it.init(a, w);
@@ -374,11 +380,12 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           if (!ok) break;
           const int first = tbl.first[slot][j];
           if (first >= 0) {
-            // consecutive window rows: one 2-D TMA box per 64-column half
+            // consecutive rows (window, or dense compressed entries): one 2-D TMA box per 64-column half
             if (plane == 0) {
+              const bool win = tbl.win[slot][j] != 0;
+              const CUtensorMap* map = is_k ? (win ? &maps.kw : &maps.kc) : (win ? &maps.vw : &maps.vc);
               mbar_expect_tx_only(full, kKVBytes);
-              for (int c = 0; c < 2; ++c)
-                tma_load_2d(dst + c * (kKVBytes / 2), is_k ? &maps.kw : &maps.vw, full, c * 64, first);
+              for (int c = 0; c < 2; ++c) tma_load_2d(dst + c * (kKVBytes / 2), map, full, c * 64, first);
             }
           } else {
             // gathered rows: a lane owns one 16-byte chunk position of a row in both
@@ -782,14 +789,18 @@ inline cudaError_t launch_attn_tc(const AttnArgs& a, int batch, cudaStream_t str
   if (!make_map_bf16_2d(&m.q, a.q, rows_q, kD, kD * 2, 64, 64)) return cudaErrorInvalidValue;
   if (!make_map_bf16_2d(&m.kw, a.kw, (uint64_t)batch * a.ring, kD, kD * 2, kTile, 64)) return cudaErrorInvalidValue;
   if (!make_map_bf16_2d(&m.vw, a.vw, (uint64_t)batch * a.ring, kD, kD * 2, kTile, 64)) return cudaErrorInvalidValue;
-  // Masked keys copy a row of their own source; with no compressed cache at all the
-  // compressed source is the window ring (row b*0 + 0), so that row is real memory.
+  // Masked keys are zero-filled with an address inside their own source; with no
+  // compressed cache at all the compressed source is the window ring, so that
+  // address is real memory.
   AttnArgs aa = a;
   if (a.kc == nullptr || a.vc == nullptr || a.nc_cap <= 0) {
     aa.kc = a.kw;
     aa.vc = a.vw;
     aa.nc_cap = 0;
   }
+  const uint64_t rows_c = aa.nc_cap > 0 ? (uint64_t)batch * aa.nc_cap : (uint64_t)batch * a.ring;
+  if (!make_map_bf16_2d(&m.kc, aa.kc, rows_c, kD, kD * 2, kTile, 64)) return cudaErrorInvalidValue;
+  if (!make_map_bf16_2d(&m.vc, aa.vc, rows_c, kD, kD * 2, kTile, 64)) return cudaErrorInvalidValue;
   const int n_items = batch * a.T * a.nsplit;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
