@@ -202,7 +202,7 @@ __device__ __forceinline__ uint32_t full_par(uint32_t n, int nst) { return (n / 
 __device__ __forceinline__ uint32_t empty_par(uint32_t n, int nst) { return ((n / nst) & 1u) ^ 1u; }
 
 struct PendingPV {
-  int valid, ob, ntiles, first;
+  int valid, ob, ntiles, first, x;   // x: parity of the group's index within its query (o_full barrier)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -217,7 +217,9 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   uint8_t* sO = sP;   // output staging: P slot 0, idle once the query's last O^T update is done
 
   __shared__ uint64_t q_full[kQSt], q_empty[kQSt], k_full[kKSt], k_empty[kKSt], v_full[kVSt], v_empty[kVSt];
-  __shared__ uint64_t s_full[2], s_free[2], p_full[kPSt], p_empty[kPSt], o_full[2], o_ready[2];
+  // o_full[ob][x]: O^T update of a group of the query in accumulator ob complete, x = parity of
+  // the group's index; two barriers let the softmax lag one group behind without phase aliasing
+  __shared__ uint64_t s_full[2], s_free[2], p_full[kPSt], p_empty[kPSt], o_full[2][2], o_ready[2];
   __shared__ uint64_t t_full[kTbl], t_empty[kTbl], mma_done;
   __shared__ KeyTable tbl;
   __shared__ uint32_t tmem_base;
@@ -236,7 +238,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     for (int s = 0; s < kVSt; ++s) { mbar_init(&v_full[s], kProdLanes); mbar_init(&v_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1); mbar_init(&s_free[s], 8);
-      mbar_init(&o_full[s], 1); mbar_init(&o_ready[s], 8);
+      mbar_init(&o_full[s][0], 1); mbar_init(&o_full[s][1], 1); mbar_init(&o_ready[s], 8);
     }
     for (int s = 0; s < kPSt; ++s) { mbar_init(&p_full[s], 8); mbar_init(&p_empty[s], 1); }
     for (int s = 0; s < kTbl; ++s) { mbar_init(&t_full[s], 32); mbar_init(&t_empty[s], kTblArrivals); }
@@ -262,7 +264,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     uint32_t G = 0, n = 0, q_next = 0;
     auto service_q = [&]() {
       if (lane != 0) return;
-      while (q_next < n && mbar_try_wait(&q_empty[q_next % kQSt], empty_par(q_next, kQSt))) {
+      while (q_next < n && mbar_test_wait(&q_empty[q_next % kQSt], empty_par(q_next, kQSt))) {
         const int qb = q_next % kQSt;
         mbar_expect_tx(&q_full[qb], kQBytes);
         for (int c = 0; c < 2; ++c)
@@ -270,12 +272,13 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         ++q_next;
       }
     };
-    // Polls `bar` while serving the Q queue; false on abort or time-out.
+    // Polls `bar` while serving the Q queue (a non-suspending test, so that a Q slot
+    // freed meanwhile is refilled at once); false on abort or time-out.
     auto wait_serving = [&](uint64_t* bar, uint32_t par) {
       const unsigned long long t0 = globaltimer();
       for (uint32_t it = 0;; ++it) {
         service_q();
-        if (mbar_try_wait(bar, par)) return true;
+        if (mbar_test_wait(bar, par)) return true;
         if ((it & 63u) == 63u) {
           if (abort_flag) return false;
           if (globaltimer() - t0 > kWaitNs) {
@@ -439,7 +442,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
       constexpr int kRing = 4;
       // S stream
       Item s_it;
-      int s_w = blockIdx.x, s_g0 = 0, s_nt = 0, s_j = 0;
+      int s_w = blockIdx.x, s_g0 = 0, s_nt = 0, s_j = 0, s_gi = 0;
       bool s_have = false, s_first = true, s_open = false;
       uint32_t Gs = 0, ns = 0, kt = 0;
       // PV stream: groups whose S^T has been issued, oldest first
@@ -459,6 +462,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           if (s_w < n_items) {
             s_have = true;
             s_first = true;
+            s_gi = 0;
             s_open = false;
             s_g0 = s_it.tile_beg;
           }
@@ -495,7 +499,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
               const bool last = s_g0 + kGT >= s_it.tile_end;
               mma_commit(&s_full[sb]);
               if (last) mma_commit(&q_empty[qb]);
-              ring[(ph + pc) % kRing] = PendingPV{1, static_cast<int>(ns % 2), s_nt, s_first ? 1 : 0};
+              ring[(ph + pc) % kRing] = PendingPV{1, static_cast<int>(ns % 2), s_nt, s_first ? 1 : 0, s_gi & 1};
+              ++s_gi;
               ++pc;
               ++Gs;
               s_first = false;
@@ -538,7 +543,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
               prog = true;
             }
             if (p_j == pv.ntiles) {
-              mma_commit(&o_full[pv.ob]);
+              mma_commit(&o_full[pv.ob][pv.x]);
               p_open = false;
               ph = (ph + 1) % kRing;
               --pc;
@@ -574,7 +579,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     const int kk = quad * 32 + lane;                  // key lane of a tile; head-dim lane of O^T
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     uint32_t G = 0, n = 0, pt = 0;
-    uint32_t ofw[2] = {0, 0};
+    uint32_t ofw[2][2] = {{0, 0}, {0, 0}};   // phases of o_full[ob][x] consumed
     bool ok = true;   // on a failed wait the warps keep the same control flow (named barriers) and skip work
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
       Item it;
@@ -601,6 +606,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
 #pragma unroll
       for (int e = 0; e < 32; ++e) lp[e] = 0.f;
       bool first = true;
+      int gi = 0, cons = 0;   // group index within the query; O^T updates consumed so far
       for (int g0 = it.tile_beg; g0 < it.tile_end; g0 += kGT, ++G) {
         const int nt = min(kGT, it.tile_end - g0);
         const bool last = g0 + kGT >= it.tile_end;
@@ -652,10 +658,17 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           if (lane == 0) resc_flag[hf] = any != 0;
         }
         named_sync_softmax();
-        // ---- O^T of the previous group of this query is complete; rescale if needed
+        // ---- O^T updates this group needs complete: two groups back (so that no o_full
+        // barrier runs two phases ahead of this thread), one back when O^T is rescaled
+        {
+          const int need = resc_flag[hf] ? gi - 1 : gi - 2;
+          while (cons <= need) {
+            ok = mbar_wait(&o_full[ob][cons & 1], ofw[ob][cons & 1] & 1u, &abort_flag) && ok;
+            ++ofw[ob][cons & 1];
+            ++cons;
+          }
+        }
         if (!first) {
-          ok = mbar_wait(&o_full[ob], full_par(ofw[ob], 1), &abort_flag) && ok;
-          ++ofw[ob];
           fence_after_sync();
           if (resc_flag[hf]) {
             uint32_t v[32];
@@ -715,10 +728,14 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[sb]);
         first = false;
+        ++gi;
         if (!last) continue;
         // ---- epilogue of the item: l = sum over key lanes; o = O^T / l
-        ok = mbar_wait(&o_full[ob], full_par(ofw[ob], 1), &abort_flag) && ok;
-        ++ofw[ob];
+        while (cons < gi) {   // every O^T update of the query
+          ok = mbar_wait(&o_full[ob][cons & 1], ofw[ob][cons & 1] & 1u, &abort_flag) && ok;
+          ++ofw[ob][cons & 1];
+          ++cons;
+        }
         fence_after_sync();
         warp_xsum32(lp, lane);
         red[hf][quad][lane] = lp[0];

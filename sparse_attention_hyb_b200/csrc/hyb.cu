@@ -328,7 +328,15 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const
   if (!attn_ffma_supported(H, D) && !(dtype == HYB_DTYPE_BF16 && attn_tc_supported(H, D, q, kc, vc, kw, vw, o)))
     return HYB_ERR_UNSUPPORTED;
   const int n_keys = (idx ? k : nc) + W;
-  const int ns = attn_splits(mode, batch, T, n_keys);
+  int ns = attn_splits(mode, batch, T, n_keys);
+  if (ns > 1 && dtype == HYB_DTYPE_BF16 && attn_tc_supported(H, D, q, kc, vc, kw, vw, o)) {
+    // the tensor-core kernel splits a query's keys at 128-key tiles: no more slices
+    // than tiles, and no empty slice
+    const int tiles = ((idx ? k : nc) + attn_tc::kTile - 1) / attn_tc::kTile + (W + attn_tc::kTile - 1) / attn_tc::kTile;
+    if (ns > tiles) ns = tiles;
+    const int per = (tiles + ns - 1) / ns;
+    ns = (tiles + per - 1) / per;
+  }
   AttnArgs a{q, q_pos, kc, vc, nc, nc_cap, r, idx, k, kw, vw, ring, W, scale, o, lse,
              nullptr, nullptr, T, H, D, ns};
   if (ns > 1) {

@@ -12,7 +12,7 @@
 //               accumulators and commits them to the ring / epilogue barriers;
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time from their lane
 //               quadrant, stage each 32 x 32 fp32 block in shared memory
-//               (128-byte swizzle, two buffers per warp) and write it with a
+//               (128-byte swizzle, four buffers per warp) and write it with a
 //               TMA tensor store, so the scores leave as whole lines.
 // Column tiles no row of the CTA can see are never loaded (causal skipping).
 #pragma once
@@ -30,7 +30,8 @@ template <int KB>  // dI = 64 * KB
 struct TcScoreSmem {
   static constexpr int kA = KB * kTcBM * 128;          // bytes of the query tile
   static constexpr int kB = KB * kTcBN * 128;          // bytes of one key tile
-  static constexpr int kC = 4 * 2 * 32 * 128;         // epilogue staging: 4 warps x 2 buffers x 32 rows x 128 B
+  static constexpr int kStg = 4;                       // staging buffers per epilogue warp
+  static constexpr int kC = 4 * kStg * 32 * 128;       // epilogue staging: 4 warps x kStg buffers x 32 rows x 128 B
   static constexpr int kTotal = kA + kTcStages * kB + kC + 1024;  // + alignment slack
 };
 
@@ -139,7 +140,7 @@ scores_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     } else if (warp >= 2) {
       // ---------------- epilogue
       const int quad = warp & 3;
-      uint8_t* stg = sC + quad * (2 * 32 * 128);
+      uint8_t* stg = sC + quad * (L::kStg * 32 * 128);
       uint32_t nst = 0;   // blocks this warp has stored
       for (int it = 0; it < my_tiles; ++it) {
         const int acc = it & 1;
@@ -153,9 +154,9 @@ scores_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kTcBN + c * 32, v);
           tmem_wait_ld();
           const int cb = col0 + c * 32;
-          if (cb >= cols) continue;   // columns no row of the CTA can see
-          uint8_t* buf = stg + (nst & 1) * (32 * 128);
-          if (nst >= 2 && lane == 0) bulk_wait_read<1>();   // the store two blocks back has read this buffer
+          if (cb >= cols || m0 + quad * 32 >= nq) continue;   // columns no row can see; rows past the chunk
+          uint8_t* buf = stg + (nst % L::kStg) * (32 * 128);
+          if (nst >= L::kStg && lane == 0) bulk_wait_read<L::kStg - 1>();   // the store kStg blocks back has read this buffer
           __syncwarp();
 #pragma unroll
           for (int e = 0; e < 8; ++e)
