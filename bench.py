@@ -166,21 +166,25 @@ def attention_flops(w, ly, q_pos: np.ndarray, n_c: int) -> float:
     return 4.0 * w.H * w.D * float((comp + win).sum())
 
 
-def source_hash() -> str:
+# Sources that define each profiled kernel (its code, helpers and launch).
+KERNEL_SOURCES = {"attention": ["attn_tc.cuh", "attn.cuh", "sm100.cuh", "common.cuh"]}
+
+
+def source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "sparse_attention_hyb_b200", "csrc", "*"))):
-        h.update(open(p, "rb").read())
+    for name in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(ROOT, "sparse_attention_hyb_b200", "csrc", name), "rb").read())
     return h.hexdigest()[:16]
 
 
 def measured_traffic(kernel: str):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was
-    taken on the current kernel sources; else None."""
+    taken on the current sources of that kernel; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(kernel)
-    if not d or d.get("source_hash") != source_hash():
+    if not d or d.get("source_hash") != source_hash(kernel):
         return None
     return d.get("dram_bytes_per_launch")
 
