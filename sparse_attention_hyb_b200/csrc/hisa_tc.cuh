@@ -2,10 +2,12 @@
 // scores only the entries of each query's selected blocks).  Within a query
 // chunk every block is chosen by many queries, so instead of one gathered dot
 // product per (query, entry) the work is regrouped per block:
-//   hisa_group_kernel      one CTA per batch: inverts the per-query block lists
-//                          (select_blocks output) into per-block lists of
-//                          (query, slot) pairs, cuts them into work items of up
-//                          to kHgQ queries, and counts each query's candidates;
+//   hisa_count_kernel,     invert the per-query block lists (select_blocks
+//   hisa_offsets_kernel,   output) into per-block lists of (query, slot) pairs:
+//   hisa_scatter_kernel    per-block counts and each query's candidate count,
+//                          list offsets and work items of up to kHgQ queries of
+//                          one block, then the scatter (all grid-wide except the
+//                          per-batch scan);
 //   hisa_block_mma_kernel  one CTA per work item: the block's 128 entry keys
 //                          (one 2-D TMA tile, 128-byte swizzle) times the
 //                          item's query rows (16-byte cp.async gather) on the
@@ -24,7 +26,7 @@ namespace hyb {
 
 constexpr int kHgQ = 32;             // queries per work item (MMA N)
 constexpr int kHgBlock = 128;        // entries per block (MMA M)
-constexpr int kHgMaxBlocks = 4096;   // blocks per batch handled by the grouping kernel
+constexpr int kHgMaxBlocks = 4096;   // blocks per batch handled by the grouping kernels
 constexpr int kHgThreads = 1024;
 
 // Work item: block g, list range [start, start + n) of the block's (query, slot) pairs.
@@ -63,43 +65,52 @@ __device__ __forceinline__ int hg_block_scan(int v, int* warp_tot, int& total) {
   return warp_tot[warp] + incl - v;
 }
 
-__global__ void __launch_bounds__(kHgThreads)
-hisa_group_kernel(const int* __restrict__ q_pos, const int* __restrict__ blk, int* __restrict__ n_cand,
-                  int* __restrict__ list, HgWork* __restrict__ work, int* __restrict__ n_work, int T_, int i0,
-                  int nq, int r, int nc, int block, int top_m, int nb, int work_cap) {
-  __shared__ int cnt[kHgMaxBlocks];
-  __shared__ int fill[kHgMaxBlocks];
-  __shared__ int warp_tot[33];
-  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int g = tid; g < nb; g += kHgThreads) cnt[g] = 0;
-  __syncthreads();
-  // ---- per-block counts; candidates per query (the valid prefix of its row)
-  for (int m = warp; m < nq; m += kHgThreads / 32) {
-    const int* bl = blk + ((size_t)b * nq + m) * top_m;
-    const int v = visible_entries(q_pos[(size_t)b * T_ + i0 + m], r, nc);
-    int n2 = 0;
-    for (int s = lane; s < top_m; s += 32) {
-      const int g = bl[s];
-      if (g >= 0 && g < nb) {
-        atomicAdd(&cnt[g], 1);
-        const int rem = v - g * block;
-        n2 += rem < block ? rem : block;
-      }
+// Clears the per-block counters (before the first chunk; later chunks find them
+// cleared by hisa_offsets_kernel).
+__global__ void hisa_zero_kernel(int* __restrict__ cnt, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) cnt[i] = 0;
+}
+
+// Warp per query row: counts the row's blocks into cnt[b][g] and writes the
+// number of candidates of the row (the valid prefix of its candidate row).
+__global__ void __launch_bounds__(256)
+hisa_count_kernel(const int* __restrict__ q_pos, const int* __restrict__ blk, int* __restrict__ n_cand,
+                  int* __restrict__ cnt, int T_, int i0, int nq, int r, int nc, int block, int top_m, int nbs) {
+  const int b = blockIdx.y, lane = threadIdx.x & 31;
+  const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (m >= nq) return;
+  const int* bl = blk + ((size_t)b * nq + m) * top_m;
+  const int v = visible_entries(q_pos[(size_t)b * T_ + i0 + m], r, nc);
+  int n2 = 0;
+  for (int s = lane; s < top_m; s += 32) {
+    const int g = bl[s];
+    if (g >= 0 && g < nbs) {
+      atomicAdd(&cnt[(size_t)b * nbs + g], 1);
+      const int rem = v - g * block;
+      n2 += rem < block ? rem : block;
     }
-    n2 = warp_sum(n2);
-    if (lane == 0) n_cand[(size_t)b * nq + m] = n2;
   }
-  __syncthreads();
-  // ---- list offsets and work offsets: each thread owns a run of consecutive blocks
+  n2 = warp_sum(n2);
+  if (lane == 0) n_cand[(size_t)b * nq + m] = n2;
+}
+
+// One CTA per batch: list offsets (fill[b][g], the scatter cursor of block g) and the
+// work items (up to kHgQ queries of one block each); clears the counts.
+__global__ void __launch_bounds__(kHgThreads)
+hisa_offsets_kernel(int* __restrict__ cnt, int* __restrict__ fill, HgWork* __restrict__ work,
+                    int* __restrict__ n_work, int nbs, int work_cap) {
+  __shared__ int warp_tot[33];
+  const int b = blockIdx.x, tid = threadIdx.x;
   constexpr int kPer = kHgMaxBlocks / kHgThreads;
   const int g0 = tid * kPer;
+  int c[kPer];
   int c_sum = 0, t_sum = 0;
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int g = g0 + i;
-    const int c = g < nb ? cnt[g] : 0;
-    c_sum += c;
-    t_sum += (c + kHgQ - 1) / kHgQ;
+    c[i] = g < nbs ? cnt[(size_t)b * nbs + g] : 0;
+    c_sum += c[i];
+    t_sum += (c[i] + kHgQ - 1) / kHgQ;
   }
   int c_tot, t_tot;
   int c_off = hg_block_scan(c_sum, warp_tot, c_tot);
@@ -108,25 +119,29 @@ hisa_group_kernel(const int* __restrict__ q_pos, const int* __restrict__ blk, in
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int g = g0 + i;
-    if (g >= nb) break;
-    const int c = cnt[g];
-    fill[g] = c_off;
-    for (int t = 0; t * kHgQ < c; ++t) {
-      const int n = c - t * kHgQ;
+    if (g >= nbs) break;
+    fill[(size_t)b * nbs + g] = c_off;
+    cnt[(size_t)b * nbs + g] = 0;
+    for (int t = 0; t * kHgQ < c[i]; ++t) {
+      const int n = c[i] - t * kHgQ;
       wb[t_off + t] = HgWork{g, c_off + t * kHgQ, n < kHgQ ? n : kHgQ, 0};
     }
-    c_off += c;
-    t_off += (c + kHgQ - 1) / kHgQ;
+    c_off += c[i];
+    t_off += (c[i] + kHgQ - 1) / kHgQ;
   }
   if (tid == 0) n_work[b] = t_tot;
-  __syncthreads();
-  // ---- scatter the (query, slot) pairs into their block's list
-  int* lb = list + (size_t)b * nq * top_m;
-  for (int p = tid; p < nq * top_m; p += kHgThreads) {
-    const int m = p / top_m, s = p % top_m;
-    const int g = blk[((size_t)b * nq + m) * top_m + s];
-    if (g >= 0 && g < nb) lb[atomicAdd(&fill[g], 1)] = p;   // p = m * top_m + s
-  }
+}
+
+// (query, slot) pairs into their block's list; p = m * top_m + s.
+__global__ void __launch_bounds__(256)
+hisa_scatter_kernel(const int* __restrict__ blk, int* __restrict__ fill, int* __restrict__ list, int nq, int top_m,
+                    int nbs) {
+  const int b = blockIdx.y;
+  const int p = blockIdx.x * 256 + threadIdx.x;
+  if (p >= nq * top_m) return;
+  const size_t base = (size_t)b * nq * top_m;
+  const int g = blk[base + p];
+  if (g >= 0 && g < nbs) list[base + atomicAdd(&fill[(size_t)b * nbs + g], 1)] = p;
 }
 
 template <int KB>  // dI = 64 * KB

@@ -45,7 +45,7 @@ struct IndexPlan {
   int nq;        // queries per chunk (per batch)
   int ldS;       // flat: score row stride; HISA: block-score row stride
   int nb;        // HISA: blocks with a representative
-  size_t off_scores, off_blk, off_ncand, off_cand, off_keys, off_list, off_work, off_nwork, total;
+  size_t off_scores, off_blk, off_ncand, off_cand, off_keys, off_list, off_work, off_nwork, off_cnt, off_fill, total;
   int work_cap;  // HISA grouped stage 2: work items per batch
   bool global_keys;
 };
@@ -76,6 +76,8 @@ IndexPlan plan_index(int dtype, int batch, int T, int nc, int k, int mode, int b
     p.off_list = off;   off += align_up((size_t)batch * p.nq * top_m * 4);
     p.off_work = off;   off += align_up((size_t)batch * p.work_cap * sizeof(HgWork));
     p.off_nwork = off;  off += align_up((size_t)batch * 4);
+    p.off_cnt = off;    off += align_up((size_t)batch * (p.nb + 1) * 4);
+    p.off_fill = off;   off += align_up((size_t)batch * (p.nb + 1) * 4);
     p.total = off;
   }
   return p;
@@ -153,8 +155,20 @@ int index_topk_impl(int batch, int T_, int dI, const void* qi, const int* q_pos,
         int* list = reinterpret_cast<int*>(ws + p.off_list);
         HgWork* work = reinterpret_cast<HgWork*>(ws + p.off_work);
         int* nwork = reinterpret_cast<int*>(ws + p.off_nwork);
-        hisa_group_kernel<<<batch, kHgThreads, 0, stream>>>(q_pos, blk, ncand, list, work, nwork, T_, i0, nq, r, nc,
-                                                            block, top_m, p.nb + 1, p.work_cap);
+        int* cnt = reinterpret_cast<int*>(ws + p.off_cnt);
+        int* fill = reinterpret_cast<int*>(ws + p.off_fill);
+        const int nbs = p.nb + 1;
+        if (i0 == 0) {
+          hisa_zero_kernel<<<(batch * nbs + 255) / 256, 256, 0, stream>>>(cnt, batch * nbs);
+          count_launch();
+        }
+        hisa_count_kernel<<<dim3((nq + 7) / 8, batch), 256, 0, stream>>>(q_pos, blk, ncand, cnt, T_, i0, nq, r, nc,
+                                                                          block, top_m, nbs);
+        hisa_offsets_kernel<<<batch, kHgThreads, 0, stream>>>(cnt, fill, work, nwork, nbs, p.work_cap);
+        hisa_scatter_kernel<<<dim3((nq * top_m + 255) / 256, batch), 256, 0, stream>>>(blk, fill, list, nq, top_m,
+                                                                                        nbs);
+        count_launch();
+        count_launch();
         count_launch();
         if ((e = launch_hisa_block_mma(qi, ic, list, work, nwork, SC, batch, T_, i0, nq, dI, nc_cap, top_m,
                                        p.work_cap, stream)) != cudaSuccess)
