@@ -95,6 +95,22 @@ cudaError_t launch_scores(const void* qi, const int* q_pos, const void* keys, fl
                           int nq, int dI, int keys_cap, int r, int nc, int div, int ldS, cudaStream_t stream) {
   const int max_cols = nc / div;
   if (max_cols <= 0) return cudaSuccess;
+  if ((nq == 1 || nq == 2) && (dI == 64 || dI == 128) && reinterpret_cast<uintptr_t>(qi) % 8 == 0 &&
+      reinterpret_cast<uintptr_t>(keys) % 8 == 0) {
+    // one or two rows per batch (decode): a streaming dot-product kernel
+    const dim3 g((max_cols + kGvKeys - 1) / kGvKeys, batch);
+    const T* q = (const T*)qi;
+    const T* k = (const T*)keys;
+    if (dI == 128) {
+      if (nq == 1) scores_gemv_kernel<T, 4, 1><<<g, 256, 0, stream>>>(q, q_pos, k, S, T_, i0, keys_cap, r, nc, div, ldS);
+      else scores_gemv_kernel<T, 4, 2><<<g, 256, 0, stream>>>(q, q_pos, k, S, T_, i0, keys_cap, r, nc, div, ldS);
+    } else {
+      if (nq == 1) scores_gemv_kernel<T, 2, 1><<<g, 256, 0, stream>>>(q, q_pos, k, S, T_, i0, keys_cap, r, nc, div, ldS);
+      else scores_gemv_kernel<T, 2, 2><<<g, 256, 0, stream>>>(q, q_pos, k, S, T_, i0, keys_cap, r, nc, div, ldS);
+    }
+    count_launch();
+    return cudaGetLastError();
+  }
   if (std::is_same<T, bf16>::value && tc_scores_supported(dI, qi, keys))
     return launch_scores_tc(qi, q_pos, keys, S, batch, T_, i0, nq, dI, keys_cap, r, nc, div, ldS, max_cols, stream);
   dim3 g((max_cols + kSB_N - 1) / kSB_N, (nq + kSB_M - 1) / kSB_M, batch);

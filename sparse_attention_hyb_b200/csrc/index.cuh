@@ -3,6 +3,7 @@
 // the path for fp32 inputs and the baseline the tensor-core scorer replaces
 // for bf16.
 #pragma once
+#include <type_traits>
 #include "common.cuh"
 #include "topk.cuh"
 
@@ -15,6 +16,88 @@ constexpr int kSB_M = 64, kSB_N = 64, kSB_K = 32;
 // visible full blocks (div = block).
 __device__ __forceinline__ int score_cols(int t, int r, int nc, int div) {
   return visible_entries(t, r, nc) / div;
+}
+
+// Same scores for chunks of one or two query rows per batch (decode): streaming
+// the keys once is the whole cost, so each warp takes 32 consecutive keys (fully
+// unrolled, so their loads are in flight together), every lane holds dI/32
+// channels of the query row(s), and one transposed warp reduction leaves key
+// j0+l's score in lane l (a coalesced 128-byte store per warp and row).
+constexpr int kGvKeys = 256;   // keys per CTA: 8 warps x 32
+
+template <int N>
+__device__ __forceinline__ void gv_xsum_step(float* v, int lane, int mask) {
+  const bool hi = (lane & mask) != 0;
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    const float send = hi ? v[i] : v[i + N / 2];
+    const float keep = hi ? v[i + N / 2] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+  }
+}
+
+template <typename T, int DPL>
+__device__ __forceinline__ void gv_load(const T* p, float (&x)[DPL]) {
+  if constexpr (std::is_same<T, float>::value) {
+    static_assert(DPL % 2 == 0, "");
+#pragma unroll
+    for (int e = 0; e < DPL; e += 2) {
+      const float2 v = *reinterpret_cast<const float2*>(p + e);
+      x[e] = v.x; x[e + 1] = v.y;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < DPL; e += 2) {
+      const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(p + e);
+      x[e] = __low2float(v); x[e + 1] = __high2float(v);
+    }
+  }
+}
+
+template <typename T, int DPL, int NQ>   // DPL = dI / 32 channels per lane; NQ query rows (1 or 2)
+__global__ void __launch_bounds__(256)
+scores_gemv_kernel(const T* __restrict__ qi, const int* __restrict__ q_pos, const T* __restrict__ keys,
+                   float* __restrict__ S, int T_, int i0, int keys_cap, int r, int nc, int div, int ldS) {
+  constexpr int dI = DPL * 32;
+  const int b = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float q[NQ][DPL];
+  int cols[NQ];
+  int maxc = 0;
+#pragma unroll
+  for (int m = 0; m < NQ; ++m) {
+    const size_t row = (size_t)b * T_ + i0 + m;
+    cols[m] = score_cols(q_pos[row], r, nc, div);
+    maxc = cols[m] > maxc ? cols[m] : maxc;
+    gv_load<T, DPL>(qi + row * dI + lane * DPL, q[m]);
+  }
+  const int j0 = blockIdx.x * kGvKeys + warp * 32;
+  if (j0 >= maxc) return;
+  const T* kb = keys + (size_t)b * keys_cap * dI + lane * DPL;
+  float part[NQ][32];
+#pragma unroll
+  for (int u = 0; u < 32; ++u) {
+    float kv[DPL];
+    if (j0 + u < maxc) {
+      gv_load<T, DPL>(kb + (size_t)(j0 + u) * dI, kv);
+    } else {
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) kv[e] = 0.f;
+    }
+#pragma unroll
+    for (int m = 0; m < NQ; ++m) {
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc = fmaf(q[m][e], kv[e], acc);
+      part[m][u] = acc;
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < NQ; ++m) {
+    gv_xsum_step<32>(part[m], lane, 16); gv_xsum_step<16>(part[m], lane, 8); gv_xsum_step<8>(part[m], lane, 4);
+    gv_xsum_step<4>(part[m], lane, 2); gv_xsum_step<2>(part[m], lane, 1);
+    const int j = j0 + lane;
+    if (j < cols[m]) S[((size_t)b * NQ + m) * ldS + j] = part[m][0];
+  }
 }
 
 // S[b, i - i0, j] = qi[b, i] . keys[b, j] for j < score_cols(row), rows i in
