@@ -5,10 +5,11 @@
 // length) consecutive scores of the row in registers as order-preserving uint32
 // keys (blocked layout: thread t owns positions [t*EPT, (t+1)*EPT)).  A 12-bit
 // radix pass (4096-bin shared histogram) finds the bin that holds the k-th
-// largest key.  The keys of that bin are compacted into shared memory (normally
-// a few hundred at most) and two more radix passes over them alone (12 and 8
-// bits) give the exact k-th key K* and how many keys equal to it are taken;
-// rows where more keys share the bin run those passes over the registers.
+// largest key.  The keys of that bin are gathered into shared memory (normally
+// a few hundred at most) and one warp runs three more radix passes over them
+// alone (8, 8 and 4 bits), which give the exact k-th key K* and how many keys
+// equal to it are taken; rows where more keys share the bin run a 12-bit and
+// an 8-bit pass over the registers.
 // Because the layout is blocked, the ordered output needs a single block-wide
 // exclusive scan of per-thread (greater-than, equal-to) counts; every thread
 // then writes its selected positions in ascending order.
@@ -100,6 +101,55 @@ __device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift, i
   __syncthreads();
 }
 
+// One warp finds the remaining 20 bits of the k-th key among the n boundary-bin
+// candidates in shared memory: three radix passes (bits 19..12, 11..4, 3..0) over a
+// 256-bin histogram of its own, warp-synchronous only; leaves prefix / remaining
+// as find_digit does.
+template <int THREADS>
+__device__ __forceinline__ void resolve_candidates_warp(RegSelSmem<THREADS>& sh, uint32_t n) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = sh.prefix, rem = sh.remaining, mask = 0xFFF00000u;
+  uint32_t* h = sh.hist;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 12 : (pass == 1 ? 4 : 0);
+    const uint32_t dmask = pass == 2 ? 0xFu : 0xFFu;
+    for (int i = lane; i < 256; i += 32) h[i] = 0u;
+    __syncwarp();
+    for (uint32_t c = lane; c < n; c += 32) {
+      const uint32_t kc = sh.cand_key[c];
+      if ((kc & mask) == prefix) atomicAdd(&h[(kc >> shift) & dmask], 1u);
+    }
+    __syncwarp();
+    uint32_t v[8], tot = 0;   // lane l owns digits 8l .. 8l+7
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { v[e] = h[lane * 8 + e]; tot += v[e]; }
+    uint32_t incl = tot;      // keys in this lane's digits and above
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t u = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += u;
+    }
+    uint32_t above = incl - tot, d = 0, nrem = 0;
+    const bool mine = above < rem && rem <= above + tot;
+    if (mine) {
+#pragma unroll
+      for (int e = 7; e >= 0; --e) {
+        if (above + v[e] >= rem) { d = lane * 8 + e; nrem = rem - above; break; }
+        above += v[e];
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    d = __shfl_sync(0xffffffffu, d, src);
+    nrem = __shfl_sync(0xffffffffu, nrem, src);
+    prefix |= d << shift;
+    rem = nrem;
+    mask |= dmask << shift;
+    __syncwarp();
+  }
+  if (lane == 0) { sh.prefix = prefix; sh.remaining = rem; }
+}
+
 // Zeroes the first `nbins` histogram bins (a multiple of 4).
 template <int THREADS>
 __device__ __forceinline__ void zero_hist(RegSelSmem<THREADS>& sh, int nbins) {
@@ -141,28 +191,18 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
   const uint32_t prefix0 = sh.prefix;
   // ---- the boundary bin's keys (their number is the bin's count)
   const uint32_t n_cand = sh.bin_count;
-  __syncthreads();   // every thread has read the histogram results before it is cleared
-  zero_hist<THREADS>(sh, kSelBins);
+  __syncthreads();   // every thread has read the histogram results before it is reused
   if (n_cand <= (uint32_t)kSelCand) {
-    // few: gather them (in any order) and resolve the low 20 bits over them alone
+    // few: gather them (in any order); one warp resolves the low 20 bits over them alone
 #pragma unroll
     for (int e = 0; e < EPT; ++e)
       if (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) sh.cand_key[atomicAdd(&sh.n_slots, 1u)] = key[e];
     __syncthreads();
-    for (uint32_t c = tid; c < n_cand; c += THREADS) atomicAdd(&sh.hist[(sh.cand_key[c] >> 8) & 0xFFFu], 1u);
+    if (tid < 32) resolve_candidates_warp<THREADS>(sh, n_cand);
     __syncthreads();
-    find_digit<THREADS>(sh, 8, kSelBins);
-    const uint32_t prefix1 = sh.prefix;
-    zero_hist<THREADS>(sh, kLastBins);
-    __syncthreads();
-    for (uint32_t c = tid; c < n_cand; c += THREADS) {
-      const uint32_t kc = sh.cand_key[c];
-      if ((kc & 0xFFFFFF00u) == prefix1) atomicAdd(&sh.hist[kc & 0xFFu], 1u);
-    }
-    __syncthreads();
-    find_digit<THREADS>(sh, 0, kLastBins);
   } else {
-    // many keys share the first digit: the same two passes over the registers
+    // many keys share the first digit: a 12-bit and an 8-bit pass over the registers
+    zero_hist<THREADS>(sh, kSelBins);
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < EPT; ++e)
@@ -221,7 +261,7 @@ __device__ __forceinline__ void select_row_reg_any(const float* __restrict__ sco
 
 // Flat rows: row (b, i) keeps the k best of its visible entries.
 template <int THREADS>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, THREADS <= 256 ? 4 : 1)
 select_flat_reg_kernel(const float* __restrict__ S, const int* __restrict__ q_pos, int* __restrict__ idx, int T_,
                        int i0, int nq, int r, int nc, int k, int ldS) {
   __shared__ RegSelSmem<THREADS> sh;
@@ -234,7 +274,7 @@ select_flat_reg_kernel(const float* __restrict__ S, const int* __restrict__ q_po
 // HISA stage 1: the partial block (if any) is always kept; the best full blocks
 // fill the other slots.  blk row: kept blocks ascending, then -1.
 template <int THREADS>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, THREADS <= 256 ? 4 : 1)
 select_blocks_reg_kernel(const float* __restrict__ SB, const int* __restrict__ q_pos, int* __restrict__ blk, int T_,
                          int i0, int nq, int r, int nc, int block, int top_m, int ldB) {
   __shared__ RegSelSmem<THREADS> sh;
@@ -256,7 +296,7 @@ select_blocks_reg_kernel(const float* __restrict__ SB, const int* __restrict__ q
 
 // HISA stage 2: the k best candidates; candidate p is entry blocks[p / B] * B + p % B.
 template <int THREADS>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, THREADS <= 256 ? 4 : 1)
 select_cand_reg_kernel(const float* __restrict__ SC, const int* __restrict__ n_cand, const int* __restrict__ blk,
                        int* __restrict__ idx, int T_, int i0, int nq, int block, int top_m, int k) {
   __shared__ RegSelSmem<THREADS> sh;
