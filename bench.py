@@ -44,7 +44,7 @@ L2_FLUSH_BYTES = 256 << 20
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU oracle sample")
@@ -267,8 +267,9 @@ def bench_prefill(S, w, steps, warmup, world, flush):
     launches = per_step * steps
     stage = np.array(stage)
     step_ms = float(stage.sum(axis=1).mean())
+    median_ms = float(np.median(stage.sum(axis=1)))
     flops = attention_flops(w, st.ly, qs["q_pos"][0].cpu().numpy(), st.n_c)
-    return st, {"step_ms": step_ms, "stage_ms": stage.mean(axis=0).tolist(), "launches": launches,
+    return st, {"step_ms": step_ms, "median_ms": median_ms, "stage_ms": stage.mean(axis=0).tolist(), "launches": launches,
                 "attn_flops": flops}
 
 
@@ -360,6 +361,51 @@ def bench_decode(S, steps, warmup, flush):
             "ms_csa": csa_ms, "ms_hca": hca_ms,
             "hbm_gbs_csa": bytes_csa / (csa_ms / 1e3) / 1e9, "hbm_gbs_hca": bytes_hca / (hca_ms / 1e3) / 1e9,
             "algorithmic_bytes_csa": bytes_csa, "algorithmic_bytes_hca": bytes_hca}
+
+
+def decode_batch(decode) -> int:
+    return C.by_name(decode["workload"]).batch
+
+
+def bench_decode_append(S, warmup, flush, n_steps=512):
+    """The fused decode-step state update for batch 64 at 128K: n_steps
+    consecutive tokens (a CSA entry every 4, an HCA entry every 128, a HISA
+    representative every 512), replayed as one CUDA graph; amortized time per step."""
+    w = C.DECODE_BS64_128K
+    A = S.abi
+    csa, hca, blk = w.layer("csa"), w.layer("hca"), 128
+    B, D, dI, ring, t0 = w.batch, w.D, w.dI, w.W, w.L
+    dt = torch.bfloat16
+    ncap, nhcap = (t0 + n_steps) // csa.r, (t0 + n_steps) // hca.r
+    kc = torch.zeros(B, ncap, D, dtype=dt, device="cuda")
+    vc, ic = torch.zeros_like(kc), torch.zeros(B, ncap, dI, dtype=dt, device="cuda")
+    kh = torch.zeros(B, nhcap, D, dtype=dt, device="cuda")
+    vh = torch.zeros_like(kh)
+    reps = torch.zeros(B, ncap // blk, dI, dtype=dt, device="cuda")
+    kw = torch.zeros(B, ring, D, dtype=dt, device="cuda")
+    vw, iw = torch.zeros_like(kw), torch.zeros(B, ring, dI, dtype=dt, device="cuda")
+    zw = torch.zeros(B, ring, dtype=torch.float32, device="cuda")
+    xk = make.normal_tensor(7, "ak", (B, D), 0.1, "bf16", "cuda")
+    xv = make.normal_tensor(7, "av", (B, D), 0.1, "bf16", "cuda")
+    xi = make.normal_tensor(7, "ai", (B, dI), 0.1, "bf16", "cuda")
+    z = make.normal_tensor(7, "az", (B,), 1.0, "f32", "cuda")
+    bc, bh = make.make_bias(w, csa, "cuda"), make.make_bias(w, hca, "cuda")
+    pos = (t0 + torch.arange(n_steps, dtype=torch.int32, device="cuda"))[:, None].repeat(1, B).contiguous()
+
+    def step(ev):
+        _rec(ev, 0)
+        for i in range(n_steps):
+            A.hyb_decode_append(xk, xv, xi, z, pos[i], kw, vw, iw, zw, bias_csa=bc, r_csa=csa.r, overlap=csa.overlap,
+                                kc=kc, vc=vc, ic=ic, bias_hca=bh, r_hca=hca.r, kc_hca=kh, vc_hca=vh, block=blk,
+                                reps=reps)
+        _rec(ev, 1)
+
+    (ms,) = graph_times(step, 1, 3, warmup, flush)
+    if A.hyb_get_device_status() != 0:
+        raise RuntimeError("device status error in the decode state update")
+    return {"batch": B, "steps_timed_together": n_steps, "us_per_step": ms * 1e3 / n_steps,
+            "what": "ring append of K, V, indexer key and logit; CSA entry every 4 tokens, HCA entry every 128, "
+                    "HISA representative every 512 (one fused launch per step)"}
 
 
 # --------------------------------------------------------------------------- the other configs
@@ -652,6 +698,11 @@ def run_ours(args, world, rank, local):
         e2e_ms, h2d, d2h = bench_e2e(S, st, max(3, args.steps // 2))
         e2e_ms = max_over_ranks(e2e_ms, world)
     decode = None if args.no_decode else bench_decode(S, args.steps, args.warmup, flush)
+    if decode is not None:
+        upd = bench_decode_append(S, args.warmup, flush)
+        decode["state_update"] = upd
+        dstep_ms = decode["ms_csa"] + decode["ms_hca"] + upd["us_per_step"] / 1e3
+        decode["tokens_per_s_csa_plus_hca_with_update"] = decode_batch(decode) / (dstep_ms / 1e3)
     extras = None
     if not args.no_extras:
         extras = {"hca_prefill_32k": bench_hca_prefill(S, st, step_ms, args.steps, args.warmup, flush, pk)}
@@ -672,7 +723,8 @@ def run_ours(args, world, rank, local):
         return
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": step_ms, "median_ms_per_step": res["median_ms"],
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "L": w.L, "T": w.T, "H": w.H, "D": w.D, "dI": w.dI, "r": 4,
                    "window_span": 8, "k": 512, "W": w.W, "parallelism": f"replicas{world}",

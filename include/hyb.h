@@ -115,6 +115,36 @@ int hyb_block_reps(int dtype, int batch, int dI, const void* ic, int nc_cap,
                    hyb_stream_t stream);
 
 /*
+ * Decode-step state update, fused (the step just before index + attend when
+ * serving: append the raw token to the window ring, emit a compressed entry
+ * every r tokens, refresh the HISA representative every `block` entries; HCA
+ * article, section "怎么压", and HISA write-up, section 02, stage 1).
+ * For each sequence b the new token is at position t = pos[b] (device int32):
+ *  - xk_new, xv_new [batch, D], xi_new [batch, dI] (nullable), z_new [batch]
+ *    (its compression logit) are written to slot t mod ring of the rings
+ *    kw, vw [batch, ring, D], iw [batch, ring, dI] (required with xi_new) and
+ *    zw [batch, ring] fp32 (the rings also serve as the attention window ring);
+ *  - when t + 1 is a multiple of r_csa (bias_csa non-null), CSA entry
+ *    j = (t+1)/r_csa - 1 of kc, vc [batch, nc_cap, D] and ic [batch, nc_cap, dI]
+ *    is written, pooled exactly as hyb_compress would from the full sequence;
+ *    when moreover j + 1 is a multiple of `block` (reps non-null), reps[b, g]
+ *    (g = (j+1)/block - 1) of reps [batch, nb_cap, dI] is recomputed as
+ *    hyb_block_reps would;
+ *  - when t + 1 is a multiple of r_hca (bias_hca non-null), HCA entry
+ *    (t+1)/r_hca - 1 of kc_hca, vc_hca [batch, nch_cap, D] is written.
+ * Requires ring >= the window lengths (2 r_csa with overlap, else r_csa; r_hca),
+ * windows <= 256, D and dI multiples of 4.  An entry index past its capacity or
+ * a negative position sets HYB_ERR_DEVICE_CHECK (read with hyb_get_device_status).
+ * Results are bit-identical to hyb_compress / hyb_block_reps on the same tokens.
+ */
+int hyb_decode_append(int dtype, int batch, int D, int dI,
+                      const void* xk_new, const void* xv_new, const void* xi_new, const float* z_new,
+                      const int* pos, void* kw, void* vw, void* iw, float* zw, int ring,
+                      const float* bias_csa, int r_csa, int overlap, void* kc, void* vc, void* ic,
+                      int nc_cap, const float* bias_hca, int r_hca, void* kc_hca, void* vc_hca,
+                      int nch_cap, int block, void* reps, int nb_cap, hyb_stream_t stream);
+
+/*
  * S2 — indexer and top-k selection (HISA write-up, sections 01 and 02; the
  * output contract of section 05 step 3: k entry indices per query).
  * Query (b, i) at position t = q_pos[b, i] sees entries j < V = min(floor((t+1)/r), nc);

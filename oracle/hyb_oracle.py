@@ -261,3 +261,66 @@ def layer_row(p: LayerParams, q_t, qi_t, t: int, kc, vc, ic, reps, kw, vw, ring:
     keys, vals = key_set(t, sel, kc, vc, kw, vw, ring, p.W)
     o, lse = attend(q_t, keys, vals, p.scale)
     return idx, round_store(o, p.dtype), round_store(lse, "f32")
+
+
+# --------------------------------------------------------------------------- decode-step state update
+
+
+class DecodeState:
+    """What one sequence keeps between decode steps: the window rings (raw K, V,
+    indexer key and compression logit of the last `ring` tokens, token s at slot
+    s mod ring) and, per layer, the compressed entries emitted so far and the
+    HISA block representatives of the full blocks."""
+
+    def __init__(self, ring: int, D: int, dI: int, layers, block: int, dtype: str):
+        self.ring, self.block, self.dtype = ring, block, dtype
+        self.length = 0
+        self.kw = np.zeros((ring, D))
+        self.vw = np.zeros((ring, D))
+        self.iw = np.zeros((ring, dI))
+        self.zw = np.zeros(ring)
+        self.layers = {p.kind: p for p in layers}
+        self.kc = {p.kind: [] for p in layers}
+        self.vc = {p.kind: [] for p in layers}
+        self.ic = []      # CSA indexer keys
+        self.reps = []    # CSA block representatives
+
+
+def _ring_view(st: DecodeState, rows: np.ndarray) -> np.ndarray:
+    """The ring's rows placed at their absolute positions 0..length-1; positions
+    that have left the ring are NaN, so a read of one would poison the result."""
+    n = st.length
+    out = np.full((n,) + rows.shape[1:], np.nan)
+    lo = max(0, n - st.ring)
+    pos = np.arange(lo, n)
+    out[pos] = rows[pos % st.ring]
+    return out
+
+
+def decode_append(st: DecodeState, k_t, v_t, i_t, z_t: float, biases) -> None:
+    """One decode step's state update for the token at position t = st.length:
+    append it to the rings; when t closes a window of a layer ((t+1) a multiple
+    of r), emit that layer's next entry with the pooling of S1 (`compress`, so
+    the same definition as over the full sequence); when a CSA entry completes a
+    block of `block` entries, add that block's representative (`block_reps`).
+    HCA article, section "怎么压" (one entry per r tokens, softmax weights plus
+    position bias); HISA write-up, section 02, stage 1 (block representatives)."""
+    t = st.length
+    slot = t % st.ring
+    st.kw[slot], st.vw[slot] = np.asarray(k_t, np.float64), np.asarray(v_t, np.float64)
+    if i_t is not None:
+        st.iw[slot] = np.asarray(i_t, np.float64)
+    st.zw[slot] = float(z_t)
+    st.length = t + 1
+    for kind, p in st.layers.items():
+        if (t + 1) % p.r:
+            continue
+        j = (t + 1) // p.r - 1
+        xs = [_ring_view(st, st.kw), _ring_view(st, st.vw)] + ([_ring_view(st, st.iw)] if kind == "csa" else [])
+        out = compress(xs, _ring_view(st, st.zw), biases[kind], p.r, p.overlap, j, j + 1, st.dtype)
+        st.kc[kind].append(out[0][0])
+        st.vc[kind].append(out[1][0])
+        if kind == "csa":
+            st.ic.append(out[2][0])
+            if st.block > 0 and (j + 1) % st.block == 0:
+                st.reps.append(block_reps(np.array(st.ic[-st.block:]), st.block, st.dtype)[0])

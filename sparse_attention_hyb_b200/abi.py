@@ -35,6 +35,10 @@ SIGNATURES = {
                               _c_ptr]),
     "hyb_block_reps": (_c_int, [_c_int, _c_int, _c_int, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_ptr,
                                 _c_int, _c_ptr]),
+    "hyb_decode_append": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr,
+                                   _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_ptr, _c_int, _c_int, _c_ptr,
+                                   _c_ptr, _c_ptr, _c_int, _c_ptr, _c_int, _c_ptr, _c_ptr, _c_int, _c_int,
+                                   _c_ptr, _c_int, _c_ptr]),
     "hyb_index_topk_workspace_size": (_c_size, [_c_int] * 10),
     "hyb_index_topk": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int,
                                 _c_int, _c_int, _c_int, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_ptr,
@@ -133,6 +137,24 @@ def hyb_block_reps(ic, block: int, g_begin: int, g_end: int, reps, stream=None):
     st = lib().hyb_block_reps(_dtype_code(ic), B, dI, _ptr(ic), nc_cap, block, g_begin, g_end, _ptr(reps),
                               reps.shape[1], _stream(stream))
     _check("hyb_block_reps", st)
+
+
+def hyb_decode_append(xk_new, xv_new, xi_new, z_new, pos, kw, vw, iw, zw,
+                      bias_csa=None, r_csa: int = 0, overlap: bool = True, kc=None, vc=None, ic=None,
+                      bias_hca=None, r_hca: int = 0, kc_hca=None, vc_hca=None, block: int = 0, reps=None,
+                      stream=None):
+    """Fused decode-step state update (see include/hyb.h): xk_new/xv_new [B, D],
+    xi_new [B, dI] or None, z_new [B] fp32, pos [B] int32; rings kw/vw [B, ring, D],
+    iw [B, ring, dI], zw [B, ring]; caches as in hyb_compress / hyb_block_reps."""
+    B, D = xk_new.shape
+    dI = xi_new.shape[1] if xi_new is not None else 0
+    st = lib().hyb_decode_append(
+        _dtype_code(xk_new), B, D, dI, _ptr(xk_new), _ptr(xv_new), _ptr(xi_new), _ptr(z_new), _ptr(pos),
+        _ptr(kw), _ptr(vw), _ptr(iw), _ptr(zw), kw.shape[1], _ptr(bias_csa), r_csa, int(bool(overlap)),
+        _ptr(kc), _ptr(vc), _ptr(ic), kc.shape[1] if kc is not None else 0, _ptr(bias_hca), r_hca, _ptr(kc_hca),
+        _ptr(vc_hca), kc_hca.shape[1] if kc_hca is not None else 0, block, _ptr(reps),
+        reps.shape[1] if reps is not None else 0, _stream(stream))
+    _check("hyb_decode_append", st)
 
 
 def hyb_index_topk_workspace_size(dtype: int, batch: int, T: int, nc: int, dI: int, k: int, mode: int,

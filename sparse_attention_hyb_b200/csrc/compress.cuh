@@ -18,16 +18,44 @@ namespace hyb {
 constexpr int kCompressWarps = 4;
 constexpr int kMaxSpan = 256;
 
-template <typename T>
-__device__ __forceinline__ void pool_rows(const T* __restrict__ x, T* __restrict__ out, int C,
-                                          int start, int span, const float* w, int lane) {
+// Window weights of one entry into w[0, span): softmax over the in-range tokens
+// (position >= 0) of (logit + bias of the position in the window); z(s) returns
+// the logit of token s.  One warp.
+template <typename ZFn>
+__device__ __forceinline__ void entry_weights(ZFn z, const float* __restrict__ bias, int start, int span, float* w,
+                                              int lane) {
+  float mx = -INFINITY;
+  for (int p = lane; p < span; p += 32) {
+    const int s = start + p;
+    const float a = s >= 0 ? z(s) + bias[p] : -INFINITY;
+    w[p] = a;
+    mx = fmaxf(mx, a);
+  }
+  mx = warp_max(mx);
+  float sum = 0.f;
+  for (int p = lane; p < span; p += 32) {
+    const float e = w[p] == -INFINITY ? 0.f : __expf(w[p] - mx);
+    w[p] = e;
+    sum += e;
+  }
+  sum = warp_sum(sum);
+  const float inv = 1.f / sum;
+  for (int p = lane; p < span; p += 32) w[p] *= inv;
+  __syncwarp();
+}
+
+// out[c] = sum_p w[p] * row(start + p)[c] over C channels (4 per lane); row(s)
+// returns the address of token s's row.  One warp.
+template <typename T, typename RowFn>
+__device__ __forceinline__ void pool_entry(RowFn row, T* __restrict__ out, int C, int start, int span, const float* w,
+                                           int lane) {
   for (int c = lane * 4; c < C; c += 128) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
     for (int p = 0; p < span; ++p) {
       const float wp = w[p];
       if (wp == 0.f) continue;  // token before the start of the sequence
-      const float4 v = load4(x + (size_t)(start + p) * C + c);
+      const float4 v = load4(row(start + p) + c);
       acc.x = fmaf(wp, v.x, acc.x);
       acc.y = fmaf(wp, v.y, acc.y);
       acc.z = fmaf(wp, v.z, acc.z);
@@ -52,32 +80,12 @@ compress_kernel(const T* __restrict__ xk, const T* __restrict__ xv, const T* __r
   const int start = overlap ? (j - 1) * r : j * r;
   const float* zb = logits + (size_t)b * L;
   float* w = wts[warp];
-
-  // Weights: softmax over the in-range tokens of the window.
-  float mx = -INFINITY;
-  for (int p = lane; p < span; p += 32) {
-    const int s = start + p;
-    const float a = s >= 0 ? zb[s] + bias[p] : -INFINITY;
-    w[p] = a;
-    mx = fmaxf(mx, a);
-  }
-  mx = warp_max(mx);
-  float sum = 0.f;
-  for (int p = lane; p < span; p += 32) {
-    const float e = w[p] == -INFINITY ? 0.f : __expf(w[p] - mx);
-    w[p] = e;
-    sum += e;
-  }
-  sum = warp_sum(sum);
-  const float inv = 1.f / sum;
-  for (int p = lane; p < span; p += 32) w[p] *= inv;
-  __syncwarp();
-
+  entry_weights([&](int s) { return zb[s]; }, bias, start, span, w, lane);
   const size_t row0 = (size_t)b * L;
   const size_t out0 = (size_t)b * nc_cap + j;
-  pool_rows(xk + row0 * D, kc + out0 * D, D, start, span, w, lane);
-  pool_rows(xv + row0 * D, vc + out0 * D, D, start, span, w, lane);
-  if (xi != nullptr) pool_rows(xi + row0 * dI, ic + out0 * dI, dI, start, span, w, lane);
+  pool_entry([&](int s) { return xk + (row0 + s) * D; }, kc + out0 * D, D, start, span, w, lane);
+  pool_entry([&](int s) { return xv + (row0 + s) * D; }, vc + out0 * D, D, start, span, w, lane);
+  if (xi != nullptr) pool_entry([&](int s) { return xi + (row0 + s) * dI; }, ic + out0 * dI, dI, start, span, w, lane);
 }
 
 template <typename T>
@@ -93,6 +101,83 @@ cudaError_t launch_compress(int batch, int L, int D, int dI, const void* xk, con
       overlap, j_begin, j_end, nc_cap);
   count_launch();
   return cudaGetLastError();
+}
+
+// Decode-step state update, fused (one warp per sequence).  The new token t =
+// pos[b] goes to slot t mod ring of the window rings (K, V, and the indexer key
+// and logit, which compression needs); when t closes a CSA window ((t + 1) is a
+// multiple of r) entry (t + 1) / r - 1 is pooled from the rings with the same
+// device functions, hence the same arithmetic, as compress_kernel; likewise an
+// HCA entry; and when the CSA entry completes a block of `block` entries, that
+// block's representative is recomputed as block_reps_kernel does.  Every window
+// lies inside the rings (span <= ring is checked on the host).
+template <typename T>
+__global__ void __launch_bounds__(32)
+decode_append_kernel(const T* __restrict__ xk_new, const T* __restrict__ xv_new, const T* __restrict__ xi_new,
+                     const float* __restrict__ z_new, const int* __restrict__ pos, T* kw, T* vw, T* iw, float* zw,
+                     int ring, int D, int dI, const float* __restrict__ bias_c, int r_c, int overlap_c, T* kc, T* vc,
+                     T* ic, int nc_cap, const float* __restrict__ bias_h, int r_h, T* kch, T* vch, int nch_cap,
+                     int block, T* reps, int nb_cap) {
+  __shared__ float w[kMaxSpan];
+  const int b = blockIdx.x, lane = threadIdx.x;
+  const int t = pos[b];
+  if (t < 0) {
+    if (lane == 0) report(HYB_ERR_DEVICE_CHECK);
+    return;
+  }
+  const size_t rb = (size_t)b * ring;
+  const size_t slot = rb + t % ring;
+  for (int c = lane * 4; c < D; c += 128) {
+    store4(kw + slot * D + c, load4(xk_new + (size_t)b * D + c));
+    store4(vw + slot * D + c, load4(xv_new + (size_t)b * D + c));
+  }
+  if (iw != nullptr)
+    for (int c = lane * 4; c < dI; c += 128) store4(iw + slot * dI + c, load4(xi_new + (size_t)b * dI + c));
+  if (lane == 0) zw[slot] = z_new[b];
+  __syncwarp();
+  auto zr = [&](int s) { return zw[rb + s % ring]; };
+  if (bias_c != nullptr && (t + 1) % r_c == 0) {
+    const int j = (t + 1) / r_c - 1;
+    if (j >= nc_cap) {
+      if (lane == 0) report(HYB_ERR_DEVICE_CHECK);
+    } else {
+      const int span = overlap_c ? 2 * r_c : r_c, start = overlap_c ? (j - 1) * r_c : j * r_c;
+      entry_weights(zr, bias_c, start, span, w, lane);
+      const size_t o = (size_t)b * nc_cap + j;
+      pool_entry([&](int s) { return kw + (rb + s % ring) * D; }, kc + o * D, D, start, span, w, lane);
+      pool_entry([&](int s) { return vw + (rb + s % ring) * D; }, vc + o * D, D, start, span, w, lane);
+      if (iw != nullptr && ic != nullptr)
+        pool_entry([&](int s) { return iw + (rb + s % ring) * dI; }, ic + o * dI, dI, start, span, w, lane);
+      __syncwarp();
+      if (reps != nullptr && ic != nullptr && block > 0 && (j + 1) % block == 0 && (j + 1) / block - 1 < nb_cap) {
+        const int g = (j + 1) / block - 1;
+        const T* src = ic + ((size_t)b * nc_cap + (size_t)g * block) * dI;
+        const float inv = 1.f / (float)block;
+        for (int c = lane * 4; c < dI; c += 128) {
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int e = 0; e < block; ++e) {
+            const float4 v = load4(src + (size_t)e * dI + c);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+          }
+          acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+          store4(reps + ((size_t)b * nb_cap + g) * dI + c, acc);
+        }
+      }
+    }
+  }
+  __syncwarp();
+  if (bias_h != nullptr && (t + 1) % r_h == 0) {
+    const int j = (t + 1) / r_h - 1;
+    if (j >= nch_cap) {
+      if (lane == 0) report(HYB_ERR_DEVICE_CHECK);
+    } else {
+      const int start = j * r_h;
+      entry_weights(zr, bias_h, start, r_h, w, lane);
+      const size_t o = (size_t)b * nch_cap + j;
+      pool_entry([&](int s) { return kw + (rb + s % ring) * D; }, kch + o * D, D, start, r_h, w, lane);
+      pool_entry([&](int s) { return vw + (rb + s % ring) * D; }, vch + o * D, D, start, r_h, w, lane);
+    }
+  }
 }
 
 // HISA block representatives: the mean of the indexer keys of a full block.

@@ -283,6 +283,45 @@ int hyb_compress(int dtype, int batch, int L, int D, int dI, const void* xk, con
   return cuda_status(e);
 }
 
+int hyb_decode_append(int dtype, int batch, int D, int dI, const void* xk_new, const void* xv_new,
+                      const void* xi_new, const float* z_new, const int* pos, void* kw, void* vw, void* iw,
+                      float* zw, int ring, const float* bias_csa, int r_csa, int overlap, void* kc, void* vc,
+                      void* ic, int nc_cap, const float* bias_hca, int r_hca, void* kc_hca, void* vc_hca,
+                      int nch_cap, int block, void* reps, int nb_cap, hyb_stream_t stream) {
+  if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
+  if (batch < 0 || D <= 0 || ring < 1) return HYB_ERR_INVALID_ARG;
+  if (batch == 0) return HYB_OK;
+  if (!xk_new || !xv_new || !z_new || !pos || !kw || !vw || !zw) return HYB_ERR_INVALID_ARG;
+  if (xi_new && (!iw || dI <= 0)) return HYB_ERR_INVALID_ARG;
+  if (D % 4 != 0 || (xi_new && dI % 4 != 0)) return HYB_ERR_UNSUPPORTED;
+  if (bias_csa) {
+    const int span = overlap ? 2 * r_csa : r_csa;
+    if (r_csa < 1 || nc_cap < 0 || !kc || !vc || (xi_new && !ic)) return HYB_ERR_INVALID_ARG;
+    if (span > ring || span > kMaxSpan) return HYB_ERR_UNSUPPORTED;
+    if (reps && (!xi_new || block < 1 || nb_cap < 0)) return HYB_ERR_INVALID_ARG;
+  }
+  if (bias_hca) {
+    if (r_hca < 1 || nch_cap < 0 || !kc_hca || !vc_hca) return HYB_ERR_INVALID_ARG;
+    if (r_hca > ring || r_hca > kMaxSpan) return HYB_ERR_UNSUPPORTED;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const void* ici = bias_csa ? ic : nullptr;
+  void* rp = bias_csa ? reps : nullptr;
+  if (dtype == HYB_DTYPE_F32) {
+    decode_append_kernel<float><<<batch, 32, 0, s>>>(
+        (const float*)xk_new, (const float*)xv_new, (const float*)xi_new, z_new, pos, (float*)kw, (float*)vw,
+        (float*)(xi_new ? iw : nullptr), zw, ring, D, dI, bias_csa, r_csa, overlap ? 1 : 0, (float*)kc, (float*)vc,
+        (float*)ici, nc_cap, bias_hca, r_hca, (float*)kc_hca, (float*)vc_hca, nch_cap, block, (float*)rp, nb_cap);
+  } else {
+    decode_append_kernel<bf16><<<batch, 32, 0, s>>>(
+        (const bf16*)xk_new, (const bf16*)xv_new, (const bf16*)xi_new, z_new, pos, (bf16*)kw, (bf16*)vw,
+        (bf16*)(xi_new ? iw : nullptr), zw, ring, D, dI, bias_csa, r_csa, overlap ? 1 : 0, (bf16*)kc, (bf16*)vc,
+        (bf16*)ici, nc_cap, bias_hca, r_hca, (bf16*)kc_hca, (bf16*)vc_hca, nch_cap, block, (bf16*)rp, nb_cap);
+  }
+  count_launch();
+  return cuda_status(cudaGetLastError());
+}
+
 int hyb_block_reps(int dtype, int batch, int dI, const void* ic, int nc_cap, int block, int g_begin,
                    int g_end, void* reps, int nb_cap, hyb_stream_t stream) {
   if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;

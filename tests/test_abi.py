@@ -49,6 +49,23 @@ def test_host_argument_checks(A):
     assert L.hyb_compress(1, 1, 1024, 4, 4, 1, 1, None, 1, 1, 200, 1, 0, 1, 1, 1, None, 1, None) == A.HYB_ERR_UNSUPPORTED
     assert L.hyb_compress(1, 1, 8, 6, 4, 1, 1, None, 1, 1, 4, 1, 0, 1, 1, 1, None, 2, None) == A.HYB_ERR_UNSUPPORTED
     assert L.hyb_block_reps(1, 1, 128, 1, 100, 128, 0, 1, 1, 1, None) == A.HYB_ERR_INVALID_ARG
+    # decode append: (dtype, batch, D, dI, xk, xv, xi, z, pos, kw, vw, iw, zw, ring, bias_c, r_c, overlap,
+    # kc, vc, ic, nc_cap, bias_h, r_h, kc_h, vc_h, nch_cap, block, reps, nb_cap, stream)
+    ok = [1, 2, 128, 128, 1, 1, 1, 1, 1, 1, 1, 1, 1, 128, 1, 4, 1, 1, 1, 1, 64, 1, 128, 1, 1, 4, 16, 1, 4, None]
+    bad = list(ok); bad[0] = 9
+    assert L.hyb_decode_append(*bad) == A.HYB_ERR_UNSUPPORTED          # dtype
+    bad = list(ok); bad[8] = None
+    assert L.hyb_decode_append(*bad) == A.HYB_ERR_INVALID_ARG          # no positions
+    bad = list(ok); bad[11] = None
+    assert L.hyb_decode_append(*bad) == A.HYB_ERR_INVALID_ARG          # indexer key without its ring
+    bad = list(ok); bad[13] = 6
+    assert L.hyb_decode_append(*bad) == A.HYB_ERR_UNSUPPORTED          # ring shorter than the 2r window
+    bad = list(ok); bad[22] = 256
+    assert L.hyb_decode_append(*bad) == A.HYB_ERR_UNSUPPORTED          # HCA window longer than the ring
+    bad = list(ok); bad[2] = 126
+    assert L.hyb_decode_append(*bad) == A.HYB_ERR_UNSUPPORTED          # D not a multiple of 4
+    bad = list(ok); bad[1] = 0
+    assert L.hyb_decode_append(*bad) == A.HYB_OK                       # empty batch: nothing to do
     # index: bad mode, missing workspace, HISA without representatives
     args = [1, 1, 16, 128, 1, 1, 1, 64, 64, 4, 8]
     assert L.hyb_index_topk(*args, 5, None, 0, 0, 0, 0, 1, None, 0, None) == A.HYB_ERR_INVALID_ARG

@@ -366,3 +366,34 @@ def test_planted_keys_are_selected_by_the_oracle():
                 assert j in idx
                 hits += 1
     assert hits > 20
+
+
+# --------------------------------------------------------------------------- decode-step state update
+
+
+def test_decode_append_token_by_token_equals_full_sequence_build():
+    """Appending a sequence one token at a time (rings of 128, a CSA entry every 4
+    tokens, an HCA entry every 128, a representative every 4 CSA entries) leaves the
+    same caches and representatives as S1 over the whole sequence, and the rings hold
+    the last 128 raw rows at slot s mod 128."""
+    rs = _rs(11)
+    L, D, dI, ring, B = 600, 16, 8, 128, 4
+    xk, xv, xi = rs.normal(size=(L, D)), rs.normal(size=(L, D)), rs.normal(size=(L, dI))
+    z = rs.normal(size=L)
+    csa = O.LayerParams("csa", 4, True, ring, 0.25, "f32")
+    hca = O.LayerParams("hca", 128, False, ring, 0.25, "f32")
+    biases = {"csa": 0.1 * rs.normal(size=8), "hca": 0.1 * rs.normal(size=128)}
+    st = O.DecodeState(ring, D, dI, (csa, hca), B, "f32")
+    for t in range(L):
+        O.decode_append(st, xk[t], xv[t], xi[t], z[t], biases)
+    kc, vc, ic = O.build_caches(csa, xk, xv, xi, z, biases["csa"])
+    kh, vh, _ = O.build_caches(hca, xk, xv, None, z, biases["hca"])
+    assert len(st.kc["csa"]) == L // 4 and len(st.kc["hca"]) == L // 128 and len(st.reps) == (L // 4) // B
+    for got, want in ((st.kc["csa"], kc), (st.vc["csa"], vc), (st.ic, ic), (st.kc["hca"], kh), (st.vc["hca"], vh),
+                      (st.reps, O.block_reps(ic, B, "f32"))):
+        got = np.array(got)
+        assert got.shape == want.shape and np.all(np.isfinite(got))
+        np.testing.assert_allclose(got, want, rtol=1e-6, atol=1e-7)
+    pos = np.arange(L - ring, L)
+    np.testing.assert_array_equal(st.kw[pos % ring], xk[pos])
+    np.testing.assert_array_equal(st.zw[pos % ring], z[pos])
