@@ -504,6 +504,40 @@ def bench_index_128k(S, steps, warmup, flush):
             "flat_ms": flat_ms, "hisa_ms": hisa_ms, "hisa_speedup": flat_ms / hisa_ms}
 
 
+def bench_index_128k_tokens(S, steps, warmup, flush):
+    """Token-level indexer (r = 1, no compression: the raw indexer keys are the
+    keys, as in DSA) for the last 1024 queries of a 128K sequence: flat top-2048
+    over all previous tokens vs HISA (128-token blocks, top-64 blocks, top-2048 of
+    their tokens) -- the setting of the pages' flat-vs-HISA comparison."""
+    w = C.PREFILL_128K
+    ly = w.layer("csa")
+    wq = C.scaled(w, T=ly.q_chunk, q_pos0=w.L - ly.q_chunk)
+    A = S.abi
+    n_c = w.L
+    ic = make.normal_tensor(w.seed, "raw_index", (1, w.L, w.dI), w.i_scale, w.dtype, "cuda")
+    reps = S.layer.block_reps(ic, n_c, ly.block)
+    qs = make.make_queries(wq, "cuda")
+    idx = torch.empty(1, wq.T, ly.k, dtype=torch.int32, device="cuda")
+    idx2 = torch.empty_like(idx)
+    wsf = torch.empty(max(256, A.hyb_index_topk_workspace_size(1, 1, wq.T, n_c, w.dI, ly.k, A.HYB_INDEX_FLAT, 0, 0,
+                                                               0)), dtype=torch.uint8, device="cuda")
+    wsh = torch.empty(max(256, A.hyb_index_topk_workspace_size(1, 1, wq.T, n_c, w.dI, ly.k, A.HYB_INDEX_HISA,
+                                                               ly.block, ly.top_m, ly.q_chunk)),
+                      dtype=torch.uint8, device="cuda")
+
+    def step(ev):
+        _rec(ev, 0)
+        A.hyb_index_topk(qs["qi"], qs["q_pos"], ic, n_c, 1, ly.k, A.HYB_INDEX_FLAT, None, 0, 0, 0, idx, wsf)
+        _rec(ev, 1)
+        A.hyb_index_topk(qs["qi"], qs["q_pos"], ic, n_c, 1, ly.k, A.HYB_INDEX_HISA, reps, ly.block, ly.top_m,
+                         ly.q_chunk, idx2, wsh)
+        _rec(ev, 2)
+
+    flat_ms, hisa_ms = graph_times(step, 2, steps, warmup, flush)
+    return {"workload": "token_index_128k_last_chunk_bf16", "queries": wq.T, "k": ly.k, "r": 1,
+            "flat_ms": flat_ms, "hisa_ms": hisa_ms, "hisa_speedup": flat_ms / hisa_ms}
+
+
 def bench_1m(S, steps, warmup, flush, pk):
     """1M-token context: S1 over the whole prefix (CSA with indexer keys, HCA, HISA
     block representatives), a batch-1 decode step (CSA with the HISA indexer, HCA)
@@ -709,6 +743,8 @@ def run_ours(args, world, rank, local):
         del st
         torch.cuda.empty_cache()
         extras["index_128k_last_chunk"] = bench_index_128k(S, args.steps, args.warmup, flush)
+        torch.cuda.empty_cache()
+        extras["token_index_128k_last_chunk"] = bench_index_128k_tokens(S, args.steps, args.warmup, flush)
         torch.cuda.empty_cache()
         extras.update(bench_1m(S, args.steps, args.warmup, flush, pk))
         extras["timing"] = "median of the timed steps, CUDA-graph replay, L2 flushed between steps"
