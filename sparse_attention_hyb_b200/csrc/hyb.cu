@@ -46,6 +46,8 @@ struct IndexPlan {
   int ldS;       // flat: score row stride; HISA: block-score row stride
   int nb;        // HISA: blocks with a representative
   size_t off_scores, off_blk, off_ncand, off_cand, off_keys, off_list, off_work, off_nwork, off_cnt, off_fill, total;
+  size_t off_cidx, off_cscore;  // flat rows longer than one register block: segment winners
+  int nseg;                     // segments per row (0: single-pass selection)
   int work_cap;  // HISA grouped stage 2: work items per batch
   bool global_keys;
 };
@@ -57,10 +59,17 @@ IndexPlan plan_index(int dtype, int batch, int T, int nc, int k, int mode, int b
   if (mode == HYB_INDEX_FLAT) {
     p.ldS = round_up(nc > 0 ? nc : 1, 4);
     p.nq = q_chunk > 0 ? (q_chunk < T ? q_chunk : T) : default_chunk(batch, T, (size_t)p.ldS * 4);
-    p.global_keys = (size_t)nc * 4 > kSmemTopkMax;
+    p.nseg = 0;
+    if (nc > kSegKeys) {
+      const int nseg = (nc + kSegKeys - 1) / kSegKeys;
+      if ((long long)nseg * k <= kSegKeys) p.nseg = nseg;
+    }
+    p.global_keys = p.nseg == 0 && (size_t)nc * 4 > kSmemTopkMax;
     size_t off = 0;
     p.off_scores = off; off += align_up((size_t)batch * p.nq * p.ldS * 4);
     p.off_keys = off;   off += p.global_keys ? align_up((size_t)batch * p.nq * p.ldS * 4) : 0;
+    p.off_cidx = off;   off += p.nseg ? align_up((size_t)batch * p.nq * p.nseg * k * 4) : 0;
+    p.off_cscore = off; off += p.nseg ? align_up((size_t)batch * p.nq * p.nseg * k * 4) : 0;
     p.total = off;
   } else {
     p.nb = nc / block;
@@ -138,6 +147,18 @@ int index_topk_impl(int batch, int T_, int dI, const void* qi, const int* q_pos,
       } else if (nc <= 1024 * kRegEPT) {
         select_flat_reg_kernel<1024><<<dim3(nq, batch), 1024, 0, stream>>>(S, q_pos, idx, T_, i0, nq, r, nc, k,
                                                                            p.ldS);
+      } else if (p.nseg > 0) {
+        int* cidx = reinterpret_cast<int*>(ws + p.off_cidx);
+        float* cscore = reinterpret_cast<float*>(ws + p.off_cscore);
+        select_flat_seg_kernel<<<dim3(nq, p.nseg, batch), 1024, 0, stream>>>(S, q_pos, cidx, cscore, T_, i0, nq, r,
+                                                                             nc, k, p.ldS, p.nseg);
+        count_launch();
+        if (p.nseg * k <= 256 * kRegEPT)
+          select_flat_merge_kernel<256><<<dim3(nq, batch), 256, 0, stream>>>(q_pos, cidx, cscore, idx, T_, i0, nq, r,
+                                                                              nc, k, p.nseg);
+        else
+          select_flat_merge_kernel<1024><<<dim3(nq, batch), 1024, 0, stream>>>(q_pos, cidx, cscore, idx, T_, i0, nq,
+                                                                                r, nc, k, p.nseg);
       } else {
         const size_t smem = p.global_keys ? 0 : (size_t)nc * 4;
         if ((e = allow_smem(select_flat_kernel, smem)) != cudaSuccess) return HYB_ERR_CUDA;

@@ -259,6 +259,61 @@ __device__ __forceinline__ void select_row_reg_any(const float* __restrict__ sco
   else select_row_reg<THREADS, kRegEPT>(scores, n, k, k_out, out, map, sh);
 }
 
+// Rows longer than one register block (kSegKeys keys): exact two-level selection.
+// Pass 1 keeps the k best of every segment of kSegKeys keys; the k best of the
+// row are among those (the order -- score descending, index ascending -- is the
+// same within a segment), so pass 2 selects the k best of the segment winners.
+// The winners are laid out segment after segment, each in ascending order, so a
+// candidate's position orders ties exactly as its entry index does.
+constexpr int kSegKeys = 1024 * kRegEPT;
+
+struct OffsetMap {
+  int lo;
+  __device__ __forceinline__ int operator()(int p) const { return lo + p; }
+};
+struct CandIdxMap {
+  const int* idx;
+  __device__ __forceinline__ int operator()(int p) const { return idx[p]; }
+};
+
+__device__ __forceinline__ int seg_len(int n, int s) {
+  const int len = n - s * kSegKeys;
+  return len < 0 ? 0 : (len > kSegKeys ? kSegKeys : len);
+}
+
+__global__ void __launch_bounds__(1024, 1)
+select_flat_seg_kernel(const float* __restrict__ S, const int* __restrict__ q_pos, int* __restrict__ cidx,
+                       float* __restrict__ cscore, int T_, int i0, int nq, int r, int nc, int k, int ldS, int nseg) {
+  __shared__ RegSelSmem<1024> sh;
+  const int m = blockIdx.x, s = blockIdx.y, b = blockIdx.z;
+  const size_t row = (size_t)b * T_ + i0 + m;
+  const int n = visible_entries(q_pos[row], r, nc);
+  const int len = seg_len(n, s);
+  if (len == 0) return;
+  int off = 0;   // candidates of the segments before this one
+  for (int u = 0; u < s; ++u) off += seg_len(n, u) < k ? seg_len(n, u) : k;
+  const int kk = len < k ? len : k;
+  const size_t crow = ((size_t)b * nq + m) * (size_t)nseg * k + off;
+  const float* srow = S + ((size_t)b * nq + m) * ldS + (size_t)s * kSegKeys;
+  select_row_reg_any<1024>(srow, len, kk, kk, cidx + crow, OffsetMap{s * kSegKeys}, sh);
+  __syncthreads();
+  for (int i = threadIdx.x; i < kk; i += 1024) cscore[crow + i] = srow[cidx[crow + i] - s * kSegKeys];
+}
+
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS, THREADS <= 256 ? 4 : 1)
+select_flat_merge_kernel(const int* __restrict__ q_pos, const int* __restrict__ cidx, const float* __restrict__ cscore,
+                         int* __restrict__ idx, int T_, int i0, int nq, int r, int nc, int k, int nseg) {
+  __shared__ RegSelSmem<THREADS> sh;
+  const int m = blockIdx.x, b = blockIdx.y;
+  const size_t row = (size_t)b * T_ + i0 + m;
+  const int n = visible_entries(q_pos[row], r, nc);
+  int total = 0;
+  for (int u = 0; u < nseg; ++u) total += seg_len(n, u) < k ? seg_len(n, u) : k;
+  const size_t crow = ((size_t)b * nq + m) * (size_t)nseg * k;
+  select_row_reg_any<THREADS>(cscore + crow, total, k, k, idx + row * k, CandIdxMap{cidx + crow}, sh);
+}
+
 // Flat rows: row (b, i) keeps the k best of its visible entries.
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS, THREADS <= 256 ? 4 : 1)
