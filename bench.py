@@ -468,6 +468,30 @@ def bench_hca_prefill(S, st, csa_step_ms, steps, warmup, flush, pk):
             "csa_plus_hca_tokens_per_s": w.T / ((csa_step_ms + ms) / 1e3)}
 
 
+def bench_compress_pc(S, st, steps, warmup, flush, pk):
+    """S1 of the 32K CSA layer with per-channel compression weights (logits [L, D]
+    for K and V, [L, dI] for the indexer keys): HBM-bound streaming pass."""
+    w, raw, A = st.w, st.raw, S.abi
+    ly = st.ly
+    span = 2 * ly.r if ly.overlap else ly.r
+    L = raw["xk"].shape[1]
+    zkv = make.normal_tensor(w.seed, "z_kv", (1, L, w.D), 1.0, "f32", "cuda")
+    zi = make.normal_tensor(w.seed, "z_i", (1, L, w.dI), 1.0, "f32", "cuda")
+    bkv = make.normal_tensor(w.seed, "b_kv", (span, w.D), w.bias_std, "f32", "cuda")
+    bi = make.normal_tensor(w.seed, "b_i", (span, w.dI), w.bias_std, "f32", "cuda")
+
+    def step(ev):
+        _rec(ev, 0)
+        A.hyb_compress_pc(raw["xk"], raw["xv"], raw["xi"], zkv, bkv, zi, bi, ly.r, ly.overlap, 0, st.n_c, st.kc, st.vc,
+                          st.ic)
+        _rec(ev, 1)
+
+    (ms,) = graph_times(step, 1, steps, warmup, flush)
+    byts = L * (2 * w.D + w.dI) * 2 + L * (w.D + w.dI) * 4 + st.n_c * (2 * w.D + w.dI) * 2
+    return {"workload": "csa_compress_per_channel_32k_bf16", "ms": ms, "algorithmic_bytes": byts,
+            "hbm_gbs": byts / (ms / 1e3) / 1e9, "frac_of_hbm": byts / (ms / 1e3) / 1e9 / pk["hbm_gbs"]}
+
+
 def bench_index_128k(S, steps, warmup, flush):
     """Indexer latency of the last query chunk of a 128K prefill (queries
     130048..131071, chunk 1024): flat top-2048 over all visible entries vs HISA
@@ -739,7 +763,8 @@ def run_ours(args, world, rank, local):
         decode["tokens_per_s_csa_plus_hca_with_update"] = decode_batch(decode) / (dstep_ms / 1e3)
     extras = None
     if not args.no_extras:
-        extras = {"hca_prefill_32k": bench_hca_prefill(S, st, step_ms, args.steps, args.warmup, flush, pk)}
+        extras = {"hca_prefill_32k": bench_hca_prefill(S, st, step_ms, args.steps, args.warmup, flush, pk),
+                  "compress_per_channel_32k": bench_compress_pc(S, st, args.steps, args.warmup, flush, pk)}
         del st
         torch.cuda.empty_cache()
         extras["index_128k_last_chunk"] = bench_index_128k(S, args.steps, args.warmup, flush)

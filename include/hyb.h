@@ -103,6 +103,21 @@ int hyb_compress(int dtype, int batch, int L, int D, int dI,
                  hyb_stream_t stream);
 
 /*
+ * S1 with per-channel compression weights (the other reading of "compression
+ * weights", HCA article, section "怎么压"): channel c of entry j is
+ * sum_i w[i, c] x[i, c], w[., c] = softmax over the window's in-range tokens of
+ * (z[i, c] + bias[p, c]), p the position in the unclipped window.  K and V use
+ * z_kv [batch, L, D] and bias_kv [span, D] (fp32); the indexer keys (xi, nullable)
+ * use z_i [batch, L, dI] and bias_i [span, dI].  Windows, layouts, capacities and
+ * requirements as for hyb_compress; logits and biases 16-byte aligned.
+ */
+int hyb_compress_pc(int dtype, int batch, int L, int D, int dI,
+                    const void* xk, const void* xv, const void* xi,
+                    const float* z_kv, const float* bias_kv, const float* z_i, const float* bias_i,
+                    int r, int overlap, int j_begin, int j_end,
+                    void* kc, void* vc, void* ic, int nc_cap, hyb_stream_t stream);
+
+/*
  * HISA stage-1 representatives (HISA write-up, section 02, stage 1: each block
  * of `block` entries is summarised by one pooled vector; the mean is used).
  * For blocks g in [g_begin, g_end): reps[b, g] = mean of ic[b, g*block ..

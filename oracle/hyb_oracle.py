@@ -131,6 +131,27 @@ def compress(xs, z, bias, r: int, overlap: bool, j_begin: int, j_end: int, dtype
     return [round_store(o, dtype) for o in outs]
 
 
+def compress_per_channel(x, z, bias, r: int, overlap: bool, j_begin: int, j_end: int, dtype: str):
+    """S1 with per-channel compression weights (the other reading of "compression
+    weights" in the HCA article, section "怎么压"): channel c of entry j is
+    sum_i w[i, c] x[i, c] with w[., c] = softmax over the window's in-range tokens
+    of (z[i, c] + bias[p, c]), p the position in the unclipped window.
+    x, z: [L, C]; bias: [span, C].  Returns [j_end - j_begin, C], rounded."""
+    span = 2 * r if overlap else r
+    x = np.asarray(x, dtype=np.float64)
+    z = np.asarray(z, dtype=np.float64)
+    bias = np.asarray(bias, dtype=np.float64)
+    out = np.empty((j_end - j_begin, x.shape[1]))
+    for j in range(j_begin, j_end):
+        start = window_start(j, r, overlap)
+        s = np.arange(max(start, 0), (j + 1) * r)
+        a = z[s] + bias[s - start]                       # [n, C]
+        e = np.exp(a - a.max(axis=0, keepdims=True))
+        w = e / e.sum(axis=0, keepdims=True)
+        out[j - j_begin] = (w * x[s]).sum(axis=0)
+    return round_store(out, dtype)
+
+
 # --------------------------------------------------------------------------- S2 indexer
 
 

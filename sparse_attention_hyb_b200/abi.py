@@ -35,6 +35,9 @@ SIGNATURES = {
                               _c_ptr]),
     "hyb_block_reps": (_c_int, [_c_int, _c_int, _c_int, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_ptr,
                                 _c_int, _c_ptr]),
+    "hyb_compress_pc": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr,
+                                 _c_ptr, _c_ptr, _c_int, _c_int, _c_int, _c_int, _c_ptr, _c_ptr, _c_ptr, _c_int,
+                                 _c_ptr]),
     "hyb_decode_append": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr,
                                    _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_ptr, _c_int, _c_int, _c_ptr,
                                    _c_ptr, _c_ptr, _c_int, _c_ptr, _c_int, _c_ptr, _c_ptr, _c_int, _c_int,
@@ -130,6 +133,18 @@ def hyb_compress(xk, xv, xi, logits, bias, r: int, overlap: bool, j_begin: int, 
                             _ptr(bias), r, int(bool(overlap)), j_begin, j_end, _ptr(kc), _ptr(vc),
                             _ptr(ic), kc.shape[1], _stream(stream))
     _check("hyb_compress", st)
+
+
+def hyb_compress_pc(xk, xv, xi, z_kv, bias_kv, z_i, bias_i, r: int, overlap: bool, j_begin: int, j_end: int,
+                    kc, vc, ic, stream=None):
+    """S1 with per-channel weights: z_kv [B, L, D], bias_kv [span, D], z_i [B, L, dI],
+    bias_i [span, dI] fp32 (see include/hyb.h)."""
+    B, L, D = xk.shape
+    dI = xi.shape[2] if xi is not None else 0
+    st = lib().hyb_compress_pc(_dtype_code(xk), B, L, D, dI, _ptr(xk), _ptr(xv), _ptr(xi), _ptr(z_kv), _ptr(bias_kv),
+                               _ptr(z_i), _ptr(bias_i), r, int(bool(overlap)), j_begin, j_end, _ptr(kc), _ptr(vc),
+                               _ptr(ic), kc.shape[1], _stream(stream))
+    _check("hyb_compress_pc", st)
 
 
 def hyb_block_reps(ic, block: int, g_begin: int, g_end: int, reps, stream=None):

@@ -88,6 +88,69 @@ compress_kernel(const T* __restrict__ xk, const T* __restrict__ xv, const T* __r
   if (xi != nullptr) pool_entry([&](int s) { return xi + (row0 + s) * dI; }, ic + out0 * dI, dI, start, span, w, lane);
 }
 
+// S1 with per-channel compression weights: channel c of entry j pools its window
+// with w[., c] = softmax over the in-range tokens of (z[s, c] + bias[p, c]).  K and
+// V share the logits z_kv [L, D] and bias_kv [span, D]; the indexer keys have
+// their own z_i [L, dI], bias_i [span, dI].  One warp per entry; a lane owns 4
+// channels and computes their softmax itself (no cross-lane reduction): one pass
+// over the window's logits for the maximum, one for the weights and the pooling.
+template <typename T>
+__device__ __forceinline__ void pool_entry_pc(const T* __restrict__ x0, const T* __restrict__ x1,
+                                              const float* __restrict__ z, const float* __restrict__ bias,
+                                              T* __restrict__ o0, T* __restrict__ o1, int C, int start, int span,
+                                              int lane) {
+  for (int c = lane * 4; c < C; c += 128) {
+    float4 mx = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    for (int p = 0; p < span; ++p) {
+      const int s = start + p;
+      if (s < 0) continue;
+      const float4 zz = *reinterpret_cast<const float4*>(z + (size_t)s * C + c);
+      const float4 bb = *reinterpret_cast<const float4*>(bias + (size_t)p * C + c);
+      mx.x = fmaxf(mx.x, zz.x + bb.x); mx.y = fmaxf(mx.y, zz.y + bb.y);
+      mx.z = fmaxf(mx.z, zz.z + bb.z); mx.w = fmaxf(mx.w, zz.w + bb.w);
+    }
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f), a0 = sum, a1 = sum;
+    for (int p = 0; p < span; ++p) {
+      const int s = start + p;
+      if (s < 0) continue;
+      const float4 zz = *reinterpret_cast<const float4*>(z + (size_t)s * C + c);
+      const float4 bb = *reinterpret_cast<const float4*>(bias + (size_t)p * C + c);
+      const float4 e = make_float4(__expf(zz.x + bb.x - mx.x), __expf(zz.y + bb.y - mx.y), __expf(zz.z + bb.z - mx.z),
+                                   __expf(zz.w + bb.w - mx.w));
+      sum.x += e.x; sum.y += e.y; sum.z += e.z; sum.w += e.w;
+      const float4 v0 = load4(x0 + (size_t)s * C + c);
+      a0.x = fmaf(e.x, v0.x, a0.x); a0.y = fmaf(e.y, v0.y, a0.y);
+      a0.z = fmaf(e.z, v0.z, a0.z); a0.w = fmaf(e.w, v0.w, a0.w);
+      if (x1 != nullptr) {
+        const float4 v1 = load4(x1 + (size_t)s * C + c);
+        a1.x = fmaf(e.x, v1.x, a1.x); a1.y = fmaf(e.y, v1.y, a1.y);
+        a1.z = fmaf(e.z, v1.z, a1.z); a1.w = fmaf(e.w, v1.w, a1.w);
+      }
+    }
+    store4(o0 + c, make_float4(a0.x / sum.x, a0.y / sum.y, a0.z / sum.z, a0.w / sum.w));
+    if (x1 != nullptr) store4(o1 + c, make_float4(a1.x / sum.x, a1.y / sum.y, a1.z / sum.z, a1.w / sum.w));
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kCompressWarps * 32)
+compress_pc_kernel(const T* __restrict__ xk, const T* __restrict__ xv, const T* __restrict__ xi,
+                   const float* __restrict__ z_kv, const float* __restrict__ bias_kv, const float* __restrict__ z_i,
+                   const float* __restrict__ bias_i, T* __restrict__ kc, T* __restrict__ vc, T* __restrict__ ic,
+                   int L, int D, int dI, int r, int overlap, int j_begin, int j_end, int nc_cap) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int j = j_begin + blockIdx.x * kCompressWarps + warp;
+  if (j >= j_end) return;
+  const int span = overlap ? 2 * r : r;
+  const int start = overlap ? (j - 1) * r : j * r;
+  const size_t row0 = (size_t)b * L, out0 = (size_t)b * nc_cap + j;
+  pool_entry_pc(xk + row0 * D, xv + row0 * D, z_kv + row0 * D, bias_kv, kc + out0 * D, vc + out0 * D, D, start, span,
+                lane);
+  if (xi != nullptr)
+    pool_entry_pc<T>(xi + row0 * dI, nullptr, z_i + row0 * dI, bias_i, ic + out0 * dI, nullptr, dI, start, span, lane);
+}
+
 template <typename T>
 cudaError_t launch_compress(int batch, int L, int D, int dI, const void* xk, const void* xv,
                             const void* xi, const float* logits, const float* bias, int r,

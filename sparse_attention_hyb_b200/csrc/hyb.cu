@@ -304,6 +304,36 @@ int hyb_compress(int dtype, int batch, int L, int D, int dI, const void* xk, con
   return cuda_status(e);
 }
 
+int hyb_compress_pc(int dtype, int batch, int L, int D, int dI, const void* xk, const void* xv, const void* xi,
+                    const float* z_kv, const float* bias_kv, const float* z_i, const float* bias_i, int r,
+                    int overlap, int j_begin, int j_end, void* kc, void* vc, void* ic, int nc_cap,
+                    hyb_stream_t stream) {
+  if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
+  if (batch < 0 || L < 0 || D <= 0 || r < 1 || j_begin < 0 || j_end < j_begin || nc_cap < j_end)
+    return HYB_ERR_INVALID_ARG;
+  if ((long long)j_end * r > L) return HYB_ERR_INVALID_ARG;
+  if (!xk || !xv || !z_kv || !bias_kv || !kc || !vc) return HYB_ERR_INVALID_ARG;
+  if (xi && (!ic || !z_i || !bias_i || dI <= 0)) return HYB_ERR_INVALID_ARG;
+  auto al = [](const void* p) { return p == nullptr || reinterpret_cast<uintptr_t>(p) % 16 == 0; };
+  const int span = overlap ? 2 * r : r;
+  if (span > kMaxSpan || D % 4 != 0 || (xi && dI % 4 != 0) || !al(z_kv) || !al(bias_kv) || !al(z_i) || !al(bias_i))
+    return HYB_ERR_UNSUPPORTED;
+  const int n = j_end - j_begin;
+  if (n == 0 || batch == 0) return HYB_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid((n + kCompressWarps - 1) / kCompressWarps, batch);
+  if (dtype == HYB_DTYPE_F32)
+    compress_pc_kernel<float><<<grid, kCompressWarps * 32, 0, s>>>(
+        (const float*)xk, (const float*)xv, (const float*)xi, z_kv, bias_kv, z_i, bias_i, (float*)kc, (float*)vc,
+        (float*)ic, L, D, dI, r, overlap ? 1 : 0, j_begin, j_end, nc_cap);
+  else
+    compress_pc_kernel<bf16><<<grid, kCompressWarps * 32, 0, s>>>(
+        (const bf16*)xk, (const bf16*)xv, (const bf16*)xi, z_kv, bias_kv, z_i, bias_i, (bf16*)kc, (bf16*)vc,
+        (bf16*)ic, L, D, dI, r, overlap ? 1 : 0, j_begin, j_end, nc_cap);
+  count_launch();
+  return cuda_status(cudaGetLastError());
+}
+
 int hyb_decode_append(int dtype, int batch, int D, int dI, const void* xk_new, const void* xv_new,
                       const void* xi_new, const float* z_new, const int* pos, void* kw, void* vw, void* iw,
                       float* zw, int ring, const float* bias_csa, int r_csa, int overlap, void* kc, void* vc,

@@ -397,3 +397,32 @@ def test_decode_append_token_by_token_equals_full_sequence_build():
     pos = np.arange(L - ring, L)
     np.testing.assert_array_equal(st.kw[pos % ring], xk[pos])
     np.testing.assert_array_equal(st.zw[pos % ring], z[pos])
+
+
+# --------------------------------------------------------------------------- per-channel compression weights
+
+
+@pytest.mark.parametrize("r,overlap", [(4, True), (128, False), (3, True)])
+def test_compress_per_channel_with_equal_channels_is_scalar_compress(r, overlap):
+    """Every channel given the same logit and bias reduces to the scalar-weight S1."""
+    rs = _rs(21)
+    L, C = 7 * r + 5, 12
+    x = rs.normal(size=(L, C))
+    z1 = rs.normal(size=L)
+    b1 = 0.3 * rs.normal(size=2 * r if overlap else r)
+    zc, bc = np.repeat(z1[:, None], C, axis=1), np.repeat(b1[:, None], C, axis=1)
+    got = O.compress_per_channel(x, zc, bc, r, overlap, 0, L // r, "f32")
+    want = O.compress([x], z1, b1, r, overlap, 0, L // r, "f32")[0]
+    np.testing.assert_allclose(got, want, rtol=1e-6, atol=1e-7)
+
+
+def test_compress_per_channel_channels_are_independent():
+    """Channel c depends only on column c of x, z and bias: each channel equals the
+    scalar S1 run on that channel alone."""
+    rs = _rs(22)
+    r, L, C = 4, 41, 5
+    x, z, b = rs.normal(size=(L, C)), rs.normal(size=(L, C)), 0.5 * rs.normal(size=(8, C))
+    got = O.compress_per_channel(x, z, b, r, True, 0, L // r, "f32")
+    for c in range(C):
+        want = O.compress([x[:, c:c + 1]], z[:, c], b[:, c], r, True, 0, L // r, "f32")[0][:, 0]
+        np.testing.assert_allclose(got[:, c], want, rtol=1e-6, atol=1e-7)

@@ -78,6 +78,43 @@ def test_compress(S, dtype, B, L, D, dI, r, overlap, j0, j1):
         assert torch.all(kc[b, :j0] == 0) and torch.all(kc[b, j1:] == 0)   # nothing outside the range
 
 
+@pytest.mark.parametrize("dtype,B,L,D,dI,r,overlap,j0,j1", [
+    ("f32", 1, 130, 64, 32, 4, True, 0, 32),
+    ("bf16", 2, 3001, 128, 128, 4, True, 0, 750),
+    ("bf16", 2, 3001, 128, 128, 4, True, 7, 301),     # ragged range
+    ("bf16", 1, 1000, 128, 0, 128, False, 0, 7),      # HCA geometry, no indexer keys
+])
+def test_compress_per_channel(S, dtype, B, L, D, dI, r, overlap, j0, j1):
+    sc = 1.0 if dtype == "f32" else 128 ** -0.5
+    span = 2 * r if overlap else r
+    xk, xv = _normal("pk", (B, L, D), sc, dtype), _normal("pv", (B, L, D), sc, dtype)
+    xi = _normal("pi", (B, L, dI), sc, dtype) if dI else None
+    zkv, bkv = _normal("pzkv", (B, L, D), 1.0, "f32"), _normal("pbkv", (span, D), 0.3, "f32")
+    zi = _normal("pzi", (B, L, dI), 1.0, "f32") if dI else None
+    bi = _normal("pbi", (span, dI), 0.3, "f32") if dI else None
+    nc = L // r
+    kc = torch.zeros(B, nc, D, dtype=xk.dtype, device=dev)
+    vc = torch.zeros_like(kc)
+    ic = torch.zeros(B, nc, dI, dtype=xk.dtype, device=dev) if dI else None
+    g = lambda t: None if t is None else t.to(dev)
+    S.abi.hyb_compress_pc(g(xk), g(xv), g(xi), g(zkv), g(bkv), g(zi), g(bi), r, overlap, j0, j1, kc, vc, ic)
+    torch.cuda.synchronize()
+    for b in range(B):
+        wants = [O.compress_per_channel(to64(xk[b]), to64(zkv[b]), to64(bkv), r, overlap, j0, j1, dtype),
+                 O.compress_per_channel(to64(xv[b]), to64(zkv[b]), to64(bkv), r, overlap, j0, j1, dtype)]
+        gots = [kc[b, j0:j1], vc[b, j0:j1]]
+        if dI:
+            wants.append(O.compress_per_channel(to64(xi[b]), to64(zi[b]), to64(bi), r, overlap, j0, j1, dtype))
+            gots.append(ic[b, j0:j1])
+        for gt, wt, nm in zip(gots, wants, "kvi"):
+            g64 = to64(gt)
+            check_close(g64, wt, dtype, f"compress_pc {nm} b={b}")
+            if dtype == "bf16":   # one bf16 ulp from the fp64 result, plus the fp32 accumulation error
+                slack = 2.0 ** -20 * max(1.0, float(np.abs(wt).max()))
+                assert np.all(np.abs(g64 - wt) <= _ulp_bf16(wt) * 1.0001 + slack), f"{nm}: more than one ulp"
+        assert torch.all(kc[b, :j0] == 0) and torch.all(kc[b, j1:] == 0)   # nothing outside the range
+
+
 def test_block_reps(S):
     B, nc, dI, blk = 2, 1000, 128, 128
     ic = _normal("ic", (B, nc, dI), 0.1, "bf16")
