@@ -492,6 +492,29 @@ def bench_compress_pc(S, st, steps, warmup, flush, pk):
             "hbm_gbs": byts / (ms / 1e3) / 1e9, "frac_of_hbm": byts / (ms / 1e3) / 1e9 / pk["hbm_gbs"]}
 
 
+def bench_real_kv(S, st, steps, warmup, flush):
+    """CSA attention at 32K under the real-K/V reading: the 512 selected entries of
+    each query stand for their 4 raw tokens each (up to 2048 raw keys + the window)."""
+    w, raw, qs, A = st.w, st.raw, st.qs, S.abi
+    ly = st.ly
+    o = torch.empty_like(qs["q"])
+    lse = torch.empty(1, w.T, w.H, dtype=torch.float32, device="cuda")
+
+    def step(ev):
+        _rec(ev, 0)
+        A.hyb_attn_fwd(qs["q"], qs["q_pos"], None, None, st.n_c, ly.r, st.idx, ly.k, raw["xk"], raw["xv"], w.W,
+                       st.scale, o, lse, A.HYB_ATTN_PREFILL | A.HYB_ATTN_REAL_KV, None)
+        _rec(ev, 1)
+
+    (ms,) = graph_times(step, 1, steps, warmup, flush)
+    t = qs["q_pos"][0].cpu().numpy().astype(np.int64)
+    keys = np.minimum(np.minimum((t + 1) // ly.r, st.n_c), ly.k) * ly.r + np.minimum(w.W, t + 1)
+    fl = 4.0 * w.H * w.D * float(keys.sum())
+    return {"workload": "csa_real_kv_attention_32k_bf16", "ms": ms, "tokens_per_s": w.T / (ms / 1e3),
+            "tflops_upper": fl / (ms / 1e3) / 1e12,
+            "note": "flops counted with every selected token (a token inside the window is attended once)"}
+
+
 def bench_index_128k(S, steps, warmup, flush):
     """Indexer latency of the last query chunk of a 128K prefill (queries
     130048..131071, chunk 1024): flat top-2048 over all visible entries vs HISA
@@ -764,7 +787,8 @@ def run_ours(args, world, rank, local):
     extras = None
     if not args.no_extras:
         extras = {"hca_prefill_32k": bench_hca_prefill(S, st, step_ms, args.steps, args.warmup, flush, pk),
-                  "compress_per_channel_32k": bench_compress_pc(S, st, args.steps, args.warmup, flush, pk)}
+                  "compress_per_channel_32k": bench_compress_pc(S, st, args.steps, args.warmup, flush, pk),
+                  "real_kv_attention_32k": bench_real_kv(S, st, args.steps, args.warmup, flush)}
         del st
         torch.cuda.empty_cache()
         extras["index_128k_last_chunk"] = bench_index_128k(S, args.steps, args.warmup, flush)

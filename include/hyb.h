@@ -63,6 +63,8 @@ enum {
 enum { HYB_DTYPE_F32 = 0, HYB_DTYPE_BF16 = 1 };
 enum { HYB_INDEX_FLAT = 0, HYB_INDEX_HISA = 1 };
 enum { HYB_ATTN_PREFILL = 0, HYB_ATTN_DECODE = 1 };
+/* Flag OR-ed into the attention mode: the "real K/V" reading of CSA (see hyb_attn_fwd). */
+enum { HYB_ATTN_REAL_KV = 2 };
 
 /* Human-readable name of a status code.  Never NULL. */
 const char* hyb_status_string(int status);
@@ -229,6 +231,13 @@ int hyb_index_topk_noalloc(int dtype, int batch, int T, int dI,
  * function.  Entries of idx outside [0, V) other than -1 are skipped and
  * reported as HYB_ERR_DEVICE_CHECK.  Scratch: `ws` of at least
  * hyb_attn_fwd_workspace_size(...) bytes (may be 0 for PREFILL).
+ * mode | HYB_ATTN_REAL_KV (CSA with idx only; bf16, H = 64, D = 128): the "real
+ * K/V" reading -- each selected entry j stands for its raw tokens jr .. jr+r-1,
+ * read from the ring, and the key set is those tokens and the window as a set
+ * of raw positions (a token the window holds is not repeated).  kc / vc are not
+ * read (may be NULL); the ring must still hold every selected token (in decode a
+ * full raw K/V cache with ring > t); a token that has left the ring is reported
+ * as HYB_ERR_DEVICE_CHECK.
  */
 size_t hyb_attn_fwd_workspace_size(int dtype, int batch, int T, int H, int D, int k,
                                    int nc, int W, int mode);

@@ -239,6 +239,26 @@ def key_set(t: int, sel: np.ndarray, kc, vc, kw, vw, ring: int, W: int):
     return keys, vals
 
 
+def real_kv_positions(t: int, sel: np.ndarray, r: int, W: int) -> np.ndarray:
+    """The "real K/V" reading of CSA attention (SURVEY reading F4; the pages'
+    block-sparse methods attend the real keys and values behind a selection):
+    each selected entry j stands for its r raw tokens jr .. jr+r-1, and the key
+    set is those tokens together with the window as a set of raw positions (a
+    token the window already holds is not repeated), ascending."""
+    sel = np.asarray(sel, dtype=np.int64)
+    sel = sel[sel >= 0]
+    toks = (sel[:, None] * r + np.arange(r)[None, :]).reshape(-1)
+    win = window_positions(t, W)
+    return np.union1d(toks, win)
+
+
+def key_set_real_kv(t: int, sel: np.ndarray, r: int, raw_k, raw_v, ring: int, W: int):
+    """Keys and values of query t under the real-K/V reading, read from a raw ring
+    holding at least positions 0 .. t (slot s mod ring)."""
+    pos = real_kv_positions(t, sel, r, W)
+    return np.asarray(raw_k)[pos % ring], np.asarray(raw_v)[pos % ring]
+
+
 # --------------------------------------------------------------------------- whole layer
 
 

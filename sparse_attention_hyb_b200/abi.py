@@ -21,6 +21,7 @@ HYB_ERR_CUDA, HYB_ERR_TIMEOUT, HYB_ERR_DEVICE_CHECK = 4, 5, 6
 HYB_DTYPE_F32, HYB_DTYPE_BF16 = 0, 1
 HYB_INDEX_FLAT, HYB_INDEX_HISA = 0, 1
 HYB_ATTN_PREFILL, HYB_ATTN_DECODE = 0, 1
+HYB_ATTN_REAL_KV = 2   # flag OR-ed into the attention mode
 
 _c_int, _c_size, _c_ptr, _c_float = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
 

@@ -22,6 +22,7 @@ struct AttnArgs {
   void* o; float* lse;
   float* part_o; float* part_lse;  // split-KV partials (nsplit > 1)
   int T, H, D, nsplit;
+  int real_kv;  // 1: each selected entry j stands for raw tokens jr .. jr+r-1, read from the ring
 };
 
 // Key u of query t's list: u < n_comp -> compressed slot u, else window position.

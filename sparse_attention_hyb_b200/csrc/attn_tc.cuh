@@ -87,11 +87,11 @@ struct Maps {
 // the window positions w0 .. w0+n_win-1.
 struct KeyList {
   int row, t, vis, n_comp, n_win, w0, comp_tiles, tiles;
-  __device__ void init(const AttnArgs& a, int row_) {
+  __device__ void init(const AttnArgs& a, int row_, bool real_kv) {
     row = row_;
     t = a.q_pos[row];
     vis = visible_entries(t, a.r, a.nc);
-    n_comp = a.idx ? a.k : vis;
+    n_comp = a.idx ? (real_kv ? a.k * a.r : a.k) : vis;
     w0 = t - a.W + 1 > 0 ? t - a.W + 1 : 0;
     n_win = a.W > 0 ? t - w0 + 1 : 0;
     comp_tiles = (n_comp + kTile - 1) / kTile;
@@ -103,10 +103,10 @@ struct KeyList {
 struct Item {
   KeyList kl;
   int split, tile_beg, tile_end;
-  __device__ void init(const AttnArgs& a, int w) {
+  __device__ void init(const AttnArgs& a, int w, bool real_kv) {
     const int row = w / a.nsplit;
     split = w % a.nsplit;
-    kl.init(a, row);
+    kl.init(a, row, real_kv);
     const int per = (kl.tiles + a.nsplit - 1) / a.nsplit;
     tile_beg = split * per;
     tile_end = min(kl.tiles, tile_beg + per);
@@ -116,21 +116,29 @@ struct Item {
 };
 
 // Indexer entry behind key kk of compressed tile `tile` (the dense range when
-// there is no indexer); -1 for window tiles and padding.  A pure load, so a
-// group's loads can all be in flight together.
-__device__ __forceinline__ int key_entry(const AttnArgs& a, const KeyList& kl, int tile, int kk) {
+// there is no indexer; with real K/V, key u is token u mod r of entry u / r);
+// -1 for window tiles and padding.  A pure load, so a group's loads can all be
+// in flight together.
+__device__ __forceinline__ int key_entry(const AttnArgs& a, const KeyList& kl, int tile, int kk, bool real_kv) {
   const int u = tile * kTile + kk;
   if (tile >= kl.comp_tiles || u >= kl.n_comp) return -1;
-  return a.idx ? __ldg(a.idx + (size_t)kl.row * a.k + u) : u;
+  if (!a.idx) return u;
+  return __ldg(a.idx + (size_t)kl.row * a.k + (real_kv ? u / a.r : u));
 }
 
 // Source of key kk of a tile: entry index (compressed, from its entry e) or ring
 // slot (window); -1 for padding / masked keys, -2 for an entry outside the
 // visible range.
-__device__ __forceinline__ int key_source(const AttnArgs& a, const KeyList& kl, int tile, int kk, int e) {
+__device__ __forceinline__ int key_source(const AttnArgs& a, const KeyList& kl, int tile, int kk, int e,
+                                          bool real_kv) {
   if (tile < kl.comp_tiles) {
     if (e < 0) return -1;
-    return e < kl.vis ? e : -2;
+    if (e >= kl.vis) return -2;
+    if (!real_kv) return e;
+    const int tok = e * a.r + (tile * kTile + kk) % a.r;   // a raw token of the entry (<= t)
+    if (tok >= kl.w0) return -1;                            // the window holds it already
+    if (tok <= kl.t - a.ring) return -2;                    // no longer in the ring
+    return tok % a.ring;
   }
   const int u = (tile - kl.comp_tiles) * kTile + kk;
   if (u >= kl.n_win) return -1;
@@ -205,6 +213,7 @@ struct PendingPV {
   int valid, ob, ntiles, first, x;   // x: parity of the group's index within its query (o_full barrier)
 };
 
+template <bool RKV>   // the real-K/V reading (a compile-time switch: no cost to the other path)
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   using namespace sm100;
@@ -291,7 +300,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     };
     for (int w = blockIdx.x; w < n_items && !abort_flag; w += gridDim.x) {
       Item it;
-      it.init(a, w);
+      it.init(a, w, RKV);
       if (it.n_tiles() == 0) continue;
       const int b = it.kl.row / a.T;
       if (lane == 0) {   // (q_next is lane 0's; the queue cannot fill while the table ring holds fewer groups)
@@ -309,14 +318,14 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
 #pragma unroll
         for (int j = 0; j < kGT; ++j)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) src[j][i] = j < nt ? key_entry(a, it.kl, g0 + j, lane + 32 * i) : -1;
+          for (int i = 0; i < 4; ++i) src[j][i] = j < nt ? key_entry(a, it.kl, g0 + j, lane + 32 * i, RKV) : -1;
         if (!wait_serving(&t_empty[slot], empty_par(G, kTbl))) break;
         bool bad = false;
 #pragma unroll
         for (int j = 0; j < kGT; ++j)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int sj = j < nt ? key_source(a, it.kl, g0 + j, lane + 32 * i, src[j][i]) : -1;
+            const int sj = j < nt ? key_source(a, it.kl, g0 + j, lane + 32 * i, src[j][i], RKV) : -1;
             bad |= sj == -2;
             src[j][i] = sj < 0 ? -1 : sj;
           }
@@ -325,12 +334,13 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         for (int j = 0; j < kGT; ++j) {
           if (j >= nt) break;
           const bool win = g0 + j >= it.kl.comp_tiles;
-          const int base = win ? b * a.ring : b * a.nc_cap;
+          const bool from_ring = win || RKV;   // real K/V: compressed keys are raw tokens of the ring
+          const int base = from_ring ? b * a.ring : b * a.nc_cap;
 #pragma unroll
           for (int i = 0; i < 4; ++i) tbl.rows[slot][j * kTile + lane + 32 * i] = src[j][i] >= 0 ? base + src[j][i] : -1;
           if (lane == 0) {
             tbl.safe[slot][j] = base;
-            tbl.win[slot][j] = win ? 1 : 0;
+            tbl.win[slot][j] = from_ring ? 1 : 0;
             int first = -1;
             if (win) {   // window positions are consecutive rows unless the ring wraps inside the tile
               const int s0 = (it.kl.w0 + (g0 + j - it.kl.comp_tiles) * kTile) % a.ring;
@@ -366,7 +376,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     }
     for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
       Item it;
-      it.init(a, w);
+      it.init(a, w, RKV);
       if (it.n_tiles() == 0) continue;
       for (int g0 = it.tile_beg; g0 < it.tile_end && ok; g0 += kGT, ++G) {
         const int nt = min(kGT, it.tile_end - g0);
@@ -456,7 +466,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         bool prog = false;
         if (!s_have) {
           for (; s_w < n_items; s_w += gridDim.x) {
-            s_it.init(a, s_w);
+            s_it.init(a, s_w, RKV);
             if (s_it.n_tiles() > 0) break;
           }
           if (s_w < n_items) {
@@ -583,7 +593,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     bool ok = true;   // on a failed wait the warps keep the same control flow (named barriers) and skip work
     for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
       Item it;
-      it.init(a, w);
+      it.init(a, w, RKV);
       const bool final_out = a.nsplit == 1;
       const size_t prow = final_out ? (size_t)it.kl.row * kH : ((size_t)it.kl.row * a.nsplit + it.split) * kH;
       if (it.n_tiles() == 0) {
@@ -823,9 +833,10 @@ inline cudaError_t launch_attn_tc(const AttnArgs& a, int batch, cudaStream_t str
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = n_items < sms ? n_items : sms;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  auto kern = a.real_kv ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<<<grid, kThreads, kSmem, stream>>>(m, aa, n_items);
+  kern<<<grid, kThreads, kSmem, stream>>>(m, aa, n_items);
   count_launch();
   return cudaGetLastError();
 }

@@ -428,7 +428,7 @@ size_t hyb_attn_fwd_workspace_size(int dtype, int batch, int T, int H, int D, in
   (void)dtype;
   if (batch <= 0 || T <= 0 || H <= 0 || D <= 0) return 0;
   const int n_keys = (k > 0 ? k : nc) + W;
-  const int ns = attn_splits(mode, batch, T, n_keys);
+  const int ns = attn_splits(mode & ~HYB_ATTN_REAL_KV, batch, T, n_keys);
   if (ns <= 1) return 0;
   const size_t rows = (size_t)batch * T * ns * H;
   return align_up(rows * D * 4) + align_up(rows * 4);
@@ -439,26 +439,32 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const
                  const void* kw, const void* vw, int ring, int W, float scale, void* o, float* lse,
                  int mode, void* ws, size_t ws_bytes, hyb_stream_t stream) {
   if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
+  const bool real_kv = (mode & HYB_ATTN_REAL_KV) != 0;
+  mode &= ~HYB_ATTN_REAL_KV;
   if (mode != HYB_ATTN_PREFILL && mode != HYB_ATTN_DECODE) return HYB_ERR_INVALID_ARG;
-  if (batch < 0 || T < 0 || H <= 0 || D <= 0 || nc < 0 || nc_cap < nc || r < 1 || W < 0 ||
-      (idx && k < 1) || ring < 1 || ring < W)
+  if (batch < 0 || T < 0 || H <= 0 || D <= 0 || nc < 0 || (!real_kv && nc_cap < nc) || r < 1 || W < 0 ||
+      (idx && k < 1) || ring < 1 || ring < W || (real_kv && !idx))
     return HYB_ERR_INVALID_ARG;
   if (batch == 0 || T == 0) return HYB_OK;
-  if (!q || !q_pos || !kw || !vw || !o || ((nc > 0) && (!kc || !vc))) return HYB_ERR_INVALID_ARG;
-  if (!attn_ffma_supported(H, D) && !(dtype == HYB_DTYPE_BF16 && attn_tc_supported(H, D, q, kc, vc, kw, vw, o)))
-    return HYB_ERR_UNSUPPORTED;
+  if (!q || !q_pos || !kw || !vw || !o || (!real_kv && (nc > 0) && (!kc || !vc))) return HYB_ERR_INVALID_ARG;
+  const bool tc = dtype == HYB_DTYPE_BF16 && attn_tc_supported(H, D, q, real_kv ? nullptr : kc,
+                                                                real_kv ? nullptr : vc, kw, vw, o);
+  if (!attn_ffma_supported(H, D) && !tc) return HYB_ERR_UNSUPPORTED;
+  if (real_kv && (!tc || (long long)k * r > (1 << 30))) return HYB_ERR_UNSUPPORTED;   // tensor-core kernel only
+  if (real_kv) kc = vc = nullptr;   // the keys come from the ring
   const int n_keys = (idx ? k : nc) + W;
   int ns = attn_splits(mode, batch, T, n_keys);
-  if (ns > 1 && dtype == HYB_DTYPE_BF16 && attn_tc_supported(H, D, q, kc, vc, kw, vw, o)) {
+  if (ns > 1 && tc) {
     // the tensor-core kernel splits a query's keys at 128-key tiles: no more slices
     // than tiles, and no empty slice
-    const int tiles = ((idx ? k : nc) + attn_tc::kTile - 1) / attn_tc::kTile + (W + attn_tc::kTile - 1) / attn_tc::kTile;
+    const int n_comp = idx ? (real_kv ? k * r : k) : nc;
+    const int tiles = (n_comp + attn_tc::kTile - 1) / attn_tc::kTile + (W + attn_tc::kTile - 1) / attn_tc::kTile;
     if (ns > tiles) ns = tiles;
     const int per = (tiles + ns - 1) / ns;
     ns = (tiles + per - 1) / per;
   }
   AttnArgs a{q, q_pos, kc, vc, nc, nc_cap, r, idx, k, kw, vw, ring, W, scale, o, lse,
-             nullptr, nullptr, T, H, D, ns};
+             nullptr, nullptr, T, H, D, ns, real_kv ? 1 : 0};
   if (ns > 1) {
     const size_t rows = (size_t)batch * T * ns * H;
     const size_t need = align_up(rows * D * 4) + align_up(rows * 4);
@@ -472,7 +478,7 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const
     if ((e = launch_attn_ffma<float>(a, batch, s)) != cudaSuccess) return HYB_ERR_CUDA;
     if (ns > 1) { attn_merge_kernel<float><<<dim3(batch * T, H), 128, 0, s>>>(a); count_launch(); }
   } else {
-    if (attn_tc_supported(H, D, q, kc, vc, kw, vw, o))
+    if (tc)
       e = launch_attn_tc(a, batch, s);
     else
       e = launch_attn_ffma<bf16>(a, batch, s);

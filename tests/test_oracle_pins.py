@@ -426,3 +426,57 @@ def test_compress_per_channel_channels_are_independent():
     for c in range(C):
         want = O.compress([x[:, c:c + 1]], z[:, c], b[:, c], r, True, 0, L // r, "f32")[0][:, 0]
         np.testing.assert_allclose(got[:, c], want, rtol=1e-6, atol=1e-7)
+
+
+# --------------------------------------------------------------------------- real K/V reading of CSA attention
+
+
+def _dense_causal(q_t, xk, xv, t, scale):
+    """Plain causal attention of query t over raw positions 0..t, one head at a time."""
+    H = q_t.shape[0]
+    o, lse = np.empty((H, xk.shape[1])), np.empty(H)
+    for h in range(H):
+        s = [float(q_t[h] @ xk[j]) * scale for j in range(t + 1)]
+        m = max(s)
+        e = [math.exp(v - m) for v in s]
+        den = sum(e)
+        o[h] = sum(e[j] * xv[j] for j in range(t + 1)) / den
+        lse[h] = m + math.log(den)
+    return o, lse
+
+
+@pytest.mark.parametrize("r,W", [(4, 8), (4, 0), (1, 3), (3, 64)])
+def test_real_kv_with_every_entry_selected_is_dense_causal_attention(r, W):
+    """Selecting every visible entry covers raw tokens 0 .. r*V-1, the window covers
+    the rest up to t: the real-K/V key set is exactly positions 0..t once each."""
+    rs = _rs(31)
+    L, H, D = 50, 3, 8
+    xk, xv, q = rs.normal(size=(L, D)), rs.normal(size=(L, D)), rs.normal(size=(L, H, D))
+    for t in (0, 3, 17, 49):
+        n_vis = (t + 1) // r
+        pos = O.real_kv_positions(t, np.arange(n_vis), r, W)
+        if r * n_vis + W >= t + 1:
+            np.testing.assert_array_equal(pos, np.arange(t + 1))
+            keys, vals = O.key_set_real_kv(t, np.arange(n_vis), r, xk, xv, L, W)
+            o, lse = O.attend(q[t], keys, vals, 0.5)
+            o2, lse2 = _dense_causal(q[t], xk, xv, t, 0.5)
+            np.testing.assert_allclose(o, o2, rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(lse, lse2, rtol=1e-12, atol=1e-12)
+
+
+def test_real_kv_positions_by_brute_force():
+    """Tokens of the selected entries, minus nothing, plus the window, as a set."""
+    rs = _rs(32)
+    for _ in range(50):
+        r, W = int(rs.integers(1, 6)), int(rs.integers(0, 20))
+        t = int(rs.integers(0, 200))
+        n_vis = (t + 1) // r
+        sel = rs.choice(max(n_vis, 1), size=min(n_vis, int(rs.integers(0, 8))), replace=False) if n_vis else []
+        sel = np.concatenate([np.asarray(sel, dtype=np.int64), [-1, -1]])
+        want = set()
+        for j in sel:
+            if j >= 0:
+                want |= set(range(j * r, j * r + r))
+        want |= set(range(max(0, t - W + 1), t + 1))
+        assert O.real_kv_positions(t, sel, r, W).tolist() == sorted(want)
+        assert all(p <= t for p in want)

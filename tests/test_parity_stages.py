@@ -273,6 +273,53 @@ def test_attention(S, dtype, B, T, H, D, nc, r, k, W, L, mode):
                                atol=1e-4 if dtype == "f32" else 1e-3)
 
 
+@pytest.mark.parametrize("B,T,nc,r,k,W,L,mode", [
+    (2, 150, 2000, 4, 96, 128, 8000, "prefill"),
+    (2, 150, 2000, 4, 96, 0, 8000, "prefill"),       # no window: the selected tokens alone
+    (1, 100, 700, 4, 512, 128, 2800, "prefill"),     # k > visible entries for many rows
+    (2, 150, 2000, 4, 96, 128, 8000, "decode"),      # split-KV schedule
+])
+def test_attention_real_kv(S, B, T, nc, r, k, W, L, mode):
+    """The real-K/V reading: selected entries attend their raw tokens (from the ring,
+    here the raw sequence), together with the window as one set of positions."""
+    H, D, dtype = 64, 128, "bf16"
+    sc = D ** -0.5
+    q = _normal("q", (B, T, H, D), sc, dtype)
+    kw, vw = _normal("kw", (B, L, D), sc, dtype), _normal("vw", (B, L, D), sc, dtype)
+    q_pos = _positions(B, T, L, 9)
+    idx = _random_sel(B, T, k, q_pos, r, nc, 10)
+    md = (S.HYB_ATTN_PREFILL if mode == "prefill" else S.HYB_ATTN_DECODE) | S.HYB_ATTN_REAL_KV
+    scale = 1.0 / math.sqrt(D)
+    o, lse = S.layer.attention(q.to(dev), q_pos.to(dev), None, None, nc, r, idx.to(dev), kw.to(dev), vw.to(dev), W,
+                               scale, md)
+    torch.cuda.synchronize()
+    want_o, want_l = [], []
+    for b in range(B):
+        kw64, vw64 = to64(kw[b]), to64(vw[b])
+        for i in range(T):
+            t = int(q_pos[b, i])
+            keys, vals = O.key_set_real_kv(t, idx[b, i].numpy(), r, kw64, vw64, L, W)
+            if len(keys) == 0:   # no key at all (no window, nothing selected yet): o = 0, lse = -inf
+                want_o.append(np.zeros((H, D)))
+                want_l.append(np.full(H, -np.inf))
+                continue
+            oo, ll = O.attend(to64(q[b, i]), keys, vals, scale)
+            want_o.append(O.round_store(oo, dtype))
+            want_l.append(ll)
+    check_close(to64(o).reshape(B * T, H, D), np.stack(want_o), dtype, f"real-K/V attention {mode}")
+    np.testing.assert_allclose(to64(lse).reshape(B * T, H), np.stack(want_l), rtol=0, atol=1e-3)
+
+
+def test_attention_real_kv_reports_tokens_outside_the_ring(S):
+    B, T, H, D, nc, k, W, ring = 1, 4, 64, 128, 250, 8, 128, 256
+    q = _normal("q", (B, T, H, D), 0.1, "bf16").to(dev)
+    kw = _normal("kw", (B, ring, D), 0.1, "bf16").to(dev)
+    q_pos = torch.full((B, T), 999, dtype=torch.int32, device=dev)
+    idx = torch.arange(k, dtype=torch.int32, device=dev).repeat(B, T, 1).contiguous()   # tokens 0..31: gone
+    S.layer.attention(q, q_pos, None, None, nc, 4, idx, kw, kw, W, 0.1, S.HYB_ATTN_PREFILL | S.HYB_ATTN_REAL_KV)
+    assert S.abi.hyb_get_device_status() == S.abi.HYB_ERR_DEVICE_CHECK
+
+
 def test_attention_reports_bad_index(S):
     B, T, H, D, nc, k, W, L = 1, 4, 64, 128, 100, 8, 128, 600
     q = _normal("q", (B, T, H, D), 0.1, "bf16").to(dev)
