@@ -65,21 +65,27 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, RegSelSmem<
   return sh.warp_off[warp] + incl - v;
 }
 
-// Finds the digit d of `nbins` bins (each thread owns nbins / THREADS of them) with
-// above(d) < remaining <= above(d) + hist[d]; sets prefix |= d << shift and
-// remaining -= above(d).
-template <int THREADS>
-__device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift, int nbins) {
-  const int bpt = nbins / THREADS;
-  uint32_t tot = 0;
-  if (bpt % 4 == 0) {
-    const uint4* h4 = reinterpret_cast<const uint4*>(sh.hist + threadIdx.x * bpt);
-    for (int e = 0; e < bpt / 4; ++e) {
-      const uint4 v = h4[e];
-      tot += v.x + v.y + v.z + v.w;
+// Finds the digit d of NBINS bins (each thread owns NBINS / THREADS consecutive bins)
+// with above(d) < remaining <= above(d) + hist[d]; sets prefix |= d << shift and
+// remaining -= above(d).  A thread keeps the sums of its groups of four bins, so the
+// owner of the digit re-reads a single group.
+template <int THREADS, int NBINS>
+__device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift) {
+  constexpr int kBpt = NBINS / THREADS;
+  static_assert(kBpt >= 1 && NBINS % THREADS == 0, "whole bins per thread");
+  constexpr int kGs = kBpt % 4 == 0 ? 4 : 1;   // bins per group
+  constexpr int kNg = kBpt / kGs;
+  const uint32_t* mine = sh.hist + threadIdx.x * kBpt;
+  uint32_t gsum[kNg], tot = 0;
+#pragma unroll
+  for (int g = 0; g < kNg; ++g) {
+    if constexpr (kGs == 4) {
+      const uint4 q = reinterpret_cast<const uint4*>(mine)[g];
+      gsum[g] = q.x + q.y + q.z + q.w;
+    } else {
+      gsum[g] = mine[g];
     }
-  } else {
-    for (int e = 0; e < bpt; ++e) tot += sh.hist[threadIdx.x * bpt + e];
+    tot += gsum[g];
   }
   const uint32_t rem = sh.remaining;
   const uint32_t prefix = sh.prefix;
@@ -87,16 +93,31 @@ __device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift, i
   const uint32_t before = block_exclusive_scan<THREADS>(tot, sh, total);
   uint32_t above = total - before - tot;    // keys in bins above this thread's range
   if (above < rem && rem <= above + tot) {
-    for (int e = bpt - 1; e >= 0; --e) {
-      const uint32_t h = sh.hist[threadIdx.x * bpt + e];
-      if (above + h >= rem) {
-        sh.prefix = prefix | ((uint32_t)(threadIdx.x * bpt + e) << shift);
-        sh.remaining = rem - above;
-        sh.bin_count = h;
-        break;
-      }
-      above += h;
+    int gsel = 0;
+    bool found = false;
+#pragma unroll
+    for (int g = kNg - 1; g >= 0; --g) {
+      if (!found && above + gsum[g] >= rem) { found = true; gsel = g; }
+      if (!found) above += gsum[g];
     }
+    uint32_t v[kGs];
+    if constexpr (kGs == 4) {
+      const uint4 q = reinterpret_cast<const uint4*>(mine)[gsel];
+      v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    } else {
+      v[0] = gsum[gsel];
+    }
+    int d = 0;
+    uint32_t h = 0, nrem = 0;
+    found = false;
+#pragma unroll
+    for (int e = kGs - 1; e >= 0; --e) {
+      if (!found && above + v[e] >= rem) { found = true; d = e; h = v[e]; nrem = rem - above; }
+      if (!found) above += v[e];
+    }
+    sh.prefix = prefix | ((uint32_t)(threadIdx.x * kBpt + gsel * kGs + d) << shift);
+    sh.remaining = nrem;
+    sh.bin_count = h;
   }
   __syncthreads();
 }
@@ -167,36 +188,54 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
   for (int i = k + tid; i < k_out; i += THREADS) out[i] = -1;
   const int base = tid * EPT;
   const int cnt = n - base < 0 ? 0 : (n - base > EPT ? EPT : n - base);
-  uint32_t key[EPT];
+  // the row's scores are loaded first; the histogram is cleared while they arrive
+  float f[EPT];
   if (cnt == EPT && (reinterpret_cast<uintptr_t>(scores + base) & 15) == 0) {
 #pragma unroll
     for (int e = 0; e < EPT; e += 4) {
-      const float4 f = *reinterpret_cast<const float4*>(scores + base + e);
-      key[e] = score_key(f.x); key[e + 1] = score_key(f.y); key[e + 2] = score_key(f.z); key[e + 3] = score_key(f.w);
+      const float4 q = *reinterpret_cast<const float4*>(scores + base + e);
+      f[e] = q.x; f[e + 1] = q.y; f[e + 2] = q.z; f[e + 3] = q.w;
     }
   } else {
 #pragma unroll
-    for (int e = 0; e < EPT; ++e) key[e] = e < cnt ? score_key(scores[base + e]) : 0u;
+    for (int e = 0; e < EPT; ++e) f[e] = e < cnt ? scores[base + e] : 0.f;
   }
   constexpr int kLastBins = 256 < THREADS ? THREADS : 256;   // 8-bit pass, at least one bin per thread
   // ---- pass 0: bits 31..20
   zero_hist<THREADS>(sh, kSelBins);
   if (tid == 0) { sh.prefix = 0; sh.remaining = (uint32_t)k; sh.n_slots = 0; }
+  uint32_t key[EPT];
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) key[e] = e < cnt ? score_key(f[e]) : 0u;
   __syncthreads();
 #pragma unroll
   for (int e = 0; e < EPT; ++e)
     if (e < cnt) atomicAdd(&sh.hist[key[e] >> 20], 1u);
   __syncthreads();
-  find_digit<THREADS>(sh, 20, kSelBins);
+  find_digit<THREADS, kSelBins>(sh, 20);
   const uint32_t prefix0 = sh.prefix;
   // ---- the boundary bin's keys (their number is the bin's count)
   const uint32_t n_cand = sh.bin_count;
   __syncthreads();   // every thread has read the histogram results before it is reused
   if (n_cand <= (uint32_t)kSelCand) {
     // few: gather them (in any order); one warp resolves the low 20 bits over them alone
+    // slots reserved once per warp: a warp scan of the per-thread counts, one atomic
+    const int lane = tid & 31;
+    uint32_t mine = 0;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) mine += (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) ? 1u : 0u;
+    uint32_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    uint32_t wbase = 0;
+    if (lane == 31 && incl > 0) wbase = atomicAdd(&sh.n_slots, incl);
+    uint32_t slot = __shfl_sync(0xffffffffu, wbase, 31) + incl - mine;
 #pragma unroll
     for (int e = 0; e < EPT; ++e)
-      if (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) sh.cand_key[atomicAdd(&sh.n_slots, 1u)] = key[e];
+      if (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) sh.cand_key[slot++] = key[e];
     __syncthreads();
     if (tid < 32) resolve_candidates_warp<THREADS>(sh, n_cand);
     __syncthreads();
@@ -208,7 +247,7 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
     for (int e = 0; e < EPT; ++e)
       if (e < cnt && (key[e] & 0xFFF00000u) == prefix0) atomicAdd(&sh.hist[(key[e] >> 8) & 0xFFFu], 1u);
     __syncthreads();
-    find_digit<THREADS>(sh, 8, kSelBins);
+    find_digit<THREADS, kSelBins>(sh, 8);
     const uint32_t prefix1 = sh.prefix;
     zero_hist<THREADS>(sh, kLastBins);
     __syncthreads();
@@ -216,7 +255,7 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
     for (int e = 0; e < EPT; ++e)
       if (e < cnt && (key[e] & 0xFFFFFF00u) == prefix1) atomicAdd(&sh.hist[key[e] & 0xFFu], 1u);
     __syncthreads();
-    find_digit<THREADS>(sh, 0, kLastBins);
+    find_digit<THREADS, kLastBins>(sh, 0);
   }
   const uint32_t kth = sh.prefix, need = sh.remaining;
   // ---- ordered output
