@@ -177,7 +177,9 @@ int hyb_decode_append(int dtype, int batch, int D, int dI,
  *   reps [batch, nb_cap, dI] with nb_cap >= floor(nc/block) (HISA only)
  *   idx [batch, T, k] int32
  * `q_chunk` is the number of queries scored per pass (a scheduling choice;
- * results do not depend on it; 0 = library default).  Scratch comes from
+ * results do not depend on it; 0 = library default: about 512 MiB of fp32
+ * scores per pass for FLAT, about 64 MiB of block scores and candidates for
+ * HISA; a smaller q_chunk shrinks the workspace).  Scratch comes from
  * `ws` (device memory, 256-byte aligned) of at least
  * hyb_index_topk_workspace_size(...) bytes.
  */

@@ -31,11 +31,14 @@ inline size_t dtype_size(int dtype) { return dtype == HYB_DTYPE_F32 ? 4 : 2; }
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA; }
 
 constexpr size_t kSmemTopkMax = 200 * 1024;  // keys staged in shared memory per row
-constexpr size_t kScoreBudget = 64ull << 20; // target bytes of one chunk of scores
+constexpr size_t kScoreBudget = 64ull << 20;      // HISA: target bytes of one chunk of block scores + candidates
+constexpr size_t kFlatScoreBudget = 512ull << 20; // flat: target bytes of one chunk of scores
 
-// Queries scored per pass so that one chunk of scores stays near kScoreBudget.
-int default_chunk(int batch, int T, size_t row_bytes) {
-  size_t rows = kScoreBudget / (row_bytes * (size_t)batch);
+// Queries scored per pass so that one chunk of scores stays near `budget` bytes.
+// Fewer, larger chunks are faster (each chunk pays two launches and their tails)
+// even where the chunk no longer fits in L2.
+int default_chunk(int batch, int T, size_t row_bytes, size_t budget) {
+  size_t rows = budget / (row_bytes * (size_t)batch);
   if (rows < 64) rows = 64;
   rows = rows / 64 * 64;
   return (int)(rows < (size_t)T ? rows : (size_t)T);
@@ -58,7 +61,7 @@ IndexPlan plan_index(int dtype, int batch, int T, int nc, int k, int mode, int b
   IndexPlan p{};
   if (mode == HYB_INDEX_FLAT) {
     p.ldS = round_up(nc > 0 ? nc : 1, 4);
-    p.nq = q_chunk > 0 ? (q_chunk < T ? q_chunk : T) : default_chunk(batch, T, (size_t)p.ldS * 4);
+    p.nq = q_chunk > 0 ? (q_chunk < T ? q_chunk : T) : default_chunk(batch, T, (size_t)p.ldS * 4, kFlatScoreBudget);
     p.nseg = 0;
     if (nc > kSegKeys) {
       const int nseg = (nc + kSegKeys - 1) / kSegKeys;
@@ -75,7 +78,7 @@ IndexPlan plan_index(int dtype, int batch, int T, int nc, int k, int mode, int b
     p.nb = nc / block;
     p.ldS = round_up(p.nb > 0 ? p.nb : 1, 4);
     const size_t cand = (size_t)top_m * block;
-    p.nq = q_chunk > 0 ? (q_chunk < T ? q_chunk : T) : default_chunk(batch, T, cand * 4 + (size_t)p.ldS * 4);
+    p.nq = q_chunk > 0 ? (q_chunk < T ? q_chunk : T) : default_chunk(batch, T, cand * 4 + (size_t)p.ldS * 4, kScoreBudget);
     size_t off = 0;
     p.off_scores = off; off += align_up((size_t)batch * p.nq * p.ldS * 4);
     p.off_blk = off;    off += align_up((size_t)batch * p.nq * top_m * 4);

@@ -53,7 +53,8 @@ scores_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int b = blockIdx.z, m0 = blockIdx.x * kTcBM, split = blockIdx.y;
+  // query tiles last first: in causal order they see the most keys
+  const int b = blockIdx.z, m0 = (int)(gridDim.x - 1 - blockIdx.x) * kTcBM, split = blockIdx.y;
 
   if (tid == 0) {
     tile_cols = 0;

@@ -353,13 +353,14 @@ select_flat_merge_kernel(const int* __restrict__ q_pos, const int* __restrict__ 
   select_row_reg_any<THREADS>(cscore + crow, total, k, k, idx + row * k, CandIdxMap{cidx + crow}, sh);
 }
 
-// Flat rows: row (b, i) keeps the k best of its visible entries.
+// Flat rows: row (b, i) keeps the k best of its visible entries.  Rows are taken
+// last first: in causal order they are the longest, so the launch ends on short rows.
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS, THREADS <= 256 ? 4 : 1)
 select_flat_reg_kernel(const float* __restrict__ S, const int* __restrict__ q_pos, int* __restrict__ idx, int T_,
                        int i0, int nq, int r, int nc, int k, int ldS) {
   __shared__ RegSelSmem<THREADS> sh;
-  const int b = blockIdx.y, m = blockIdx.x;
+  const int b = blockIdx.y, m = nq - 1 - (int)blockIdx.x;
   const size_t row = (size_t)b * T_ + i0 + m;
   const int n = visible_entries(q_pos[row], r, nc);
   select_row_reg_any<THREADS>(S + ((size_t)b * nq + m) * ldS, n, k, k, idx + row * k, IdentityMap{}, sh);
