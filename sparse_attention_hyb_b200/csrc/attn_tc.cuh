@@ -459,7 +459,7 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
       PendingPV ring[kRing];
       int ph = 0, pc = 0, p_j = 0;
       bool p_open = false;
-      uint32_t vt = 0, pt = 0, ordy[2] = {0, 0};
+      uint32_t vt = 0, pt = 0, pg = 0;   // pg: groups whose O^T update was opened
       uint32_t idle = 0;
       unsigned long long idle_t0 = 0;
       for (;;) {
@@ -527,8 +527,8 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         }
         if (pc > 0) {
           const PendingPV pv = ring[ph];
-          if (!p_open && mbar_test_wait(&o_ready[pv.ob], full_par(ordy[pv.ob], 1))) {
-            ++ordy[pv.ob];
+          if (!p_open && mbar_test_wait(&o_ready[pg & 1], full_par(pg, 2))) {
+            ++pg;
             p_open = true;
             p_j = 0;
             prog = true;
@@ -697,7 +697,10 @@ attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         }
         fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&o_ready[ob]);
+        // by the parity of the group's global index: the arrival for group G + 2 needs the O^T
+        // update of group G (the wait above, or the previous query's epilogue), so the issuer
+        // has consumed this barrier's previous phase before the next one completes
+        if (lane == 0) mbar_arrive(&o_ready[G & 1]);
         // ---- pass B: probabilities into P^T
         const float* mu = m_use + hf * 32;
 #pragma unroll 1
