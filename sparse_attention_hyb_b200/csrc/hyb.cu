@@ -113,6 +113,19 @@ cudaError_t launch_scores(const void* qi, const int* q_pos, const void* keys, fl
     const dim3 g((max_cols + kGvKeys - 1) / kGvKeys, batch);
     const T* q = (const T*)qi;
     const T* k = (const T*)keys;
+    if constexpr (std::is_same<T, bf16>::value) {
+      if (reinterpret_cast<uintptr_t>(qi) % 16 == 0 && reinterpret_cast<uintptr_t>(keys) % 16 == 0) {
+        if (dI == 128) {
+          if (nq == 1) scores_gemv16_kernel<16, 1><<<g, 256, 0, stream>>>(q, q_pos, k, S, T_, i0, keys_cap, r, nc, div, ldS);
+          else scores_gemv16_kernel<16, 2><<<g, 256, 0, stream>>>(q, q_pos, k, S, T_, i0, keys_cap, r, nc, div, ldS);
+        } else {
+          if (nq == 1) scores_gemv16_kernel<8, 1><<<g, 256, 0, stream>>>(q, q_pos, k, S, T_, i0, keys_cap, r, nc, div, ldS);
+          else scores_gemv16_kernel<8, 2><<<g, 256, 0, stream>>>(q, q_pos, k, S, T_, i0, keys_cap, r, nc, div, ldS);
+        }
+        count_launch();
+        return cudaGetLastError();
+      }
+    }
     if (dI == 128) {
       if (nq == 1) scores_gemv_kernel<T, 4, 1><<<g, 256, 0, stream>>>(q, q_pos, k, S, T_, i0, keys_cap, r, nc, div, ldS);
       else scores_gemv_kernel<T, 4, 2><<<g, 256, 0, stream>>>(q, q_pos, k, S, T_, i0, keys_cap, r, nc, div, ldS);

@@ -100,6 +100,72 @@ scores_gemv_kernel(const T* __restrict__ qi, const int* __restrict__ q_pos, cons
   }
 }
 
+// bf16 variant of the same scores with 16-byte loads: LPK = dI / 8 lanes hold one
+// key row, so each load instruction of a warp covers 32 / LPK keys and a warp's 32
+// keys take LPK loads per lane, all in flight together.  The transposed reduction
+// over the LPK lanes of a key leaves key j0 + (l % LPK) * (32 / LPK) + l / LPK in
+// lane l (the warp's 32 scores in one 128-byte segment).
+// Eight bf16 (a 16-byte vector, lowest address first) to fp32: a bf16 is the upper
+// half of the fp32 with the same value.
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = __uint_as_float(w[e] << 16);
+    f[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+  }
+}
+
+template <int LPK, int NQ>
+__global__ void __launch_bounds__(256)
+scores_gemv16_kernel(const bf16* __restrict__ qi, const int* __restrict__ q_pos, const bf16* __restrict__ keys,
+                     float* __restrict__ S, int T_, int i0, int keys_cap, int r, int nc, int div, int ldS) {
+  constexpr int dI = LPK * 8, KPI = 32 / LPK;
+  const int b = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane % LPK, kofs = lane / LPK;
+  float q[NQ][8];
+  int cols[NQ];
+  int maxc = 0;
+#pragma unroll
+  for (int m = 0; m < NQ; ++m) {
+    const size_t row = (size_t)b * T_ + i0 + m;
+    cols[m] = score_cols(q_pos[row], r, nc, div);
+    maxc = cols[m] > maxc ? cols[m] : maxc;
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(qi + row * dI + sub * 8)), q[m]);
+  }
+  const int j0 = blockIdx.x * kGvKeys + warp * 32;
+  if (j0 >= maxc) return;
+  const bf16* kb = keys + (size_t)b * keys_cap * dI + sub * 8;
+  uint4 raw[LPK];
+#pragma unroll
+  for (int i = 0; i < LPK; ++i) {
+    const int j = j0 + i * KPI + kofs;
+    raw[i] = j < maxc ? __ldg(reinterpret_cast<const uint4*>(kb + (size_t)j * dI)) : make_uint4(0, 0, 0, 0);
+  }
+  float part[NQ][LPK];
+#pragma unroll
+  for (int i = 0; i < LPK; ++i) {
+    float kv[8];
+    bf16x8_to_f32(raw[i], kv);
+#pragma unroll
+    for (int m = 0; m < NQ; ++m) {
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc = fmaf(q[m][e], kv[e], acc);
+      part[m][i] = acc;
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < NQ; ++m) {
+    if constexpr (LPK == 16) gv_xsum_step<16>(part[m], lane, 8);
+    gv_xsum_step<8>(part[m], lane, 4);
+    gv_xsum_step<4>(part[m], lane, 2);
+    gv_xsum_step<2>(part[m], lane, 1);
+    const int j = j0 + sub * KPI + kofs;
+    if (j < cols[m]) S[((size_t)b * NQ + m) * ldS + j] = part[m][0];
+  }
+}
+
 // S[b, i - i0, j] = qi[b, i] . keys[b, j] for j < score_cols(row), rows i in
 // [i0, i0 + nq).  keys: [batch, keys_cap, dI].  Output row stride ldS.
 // Tiles whose columns are all invisible to every row of the tile are skipped.
