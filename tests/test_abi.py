@@ -90,4 +90,7 @@ def test_workspace_sizes(A):
     hisa = f(1, 1, 131072, 32768, 128, 2048, A.HYB_INDEX_HISA, 128, 64, 1024)
     assert hisa >= 1024 * 64 * 128 * 4
     assert A.hyb_attn_fwd_workspace_size(1, 1, 32768, 64, 128, 512, 8192, 128, A.HYB_ATTN_PREFILL) == 0
-    assert A.hyb_attn_fwd_workspace_size(1, 64, 1, 64, 128, 512, 32768, 128, A.HYB_ATTN_DECODE) > 0
+    # decode splits a query's keys (partials in the workspace) only while fewer than half
+    # of the 148 SMs would hold a query: one sequence splits, 64 do not
+    assert A.hyb_attn_fwd_workspace_size(1, 1, 1, 64, 128, 512, 32768, 128, A.HYB_ATTN_DECODE) > 0
+    assert A.hyb_attn_fwd_workspace_size(1, 64, 1, 64, 128, 512, 32768, 128, A.HYB_ATTN_DECODE) == 0
