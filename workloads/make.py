@@ -120,6 +120,9 @@ def plant_prefill(w: Workload, ly: LayerSpec, raw: Dict[str, torch.Tensor],
             continue
         i_min = max(0, first_t - w.q_pos0)
         rows = (i_min + (picks[p] * (w.T - i_min)).to(torch.int64)).clamp(max=w.T - 1)
+        # each picked row once: a row picked twice would get two different correlated
+        # values, and which write of a repeated index lands is unspecified on a GPU
+        rows = torch.unique(rows)
         for b in range(w.batch):
             q64 = qi[b, rows].to(torch.float64)
             qi[b, rows] = to_storage(_correlated_query(w, q64, u[p], p, device), w.dtype)
