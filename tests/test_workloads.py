@@ -1,7 +1,9 @@
 """The seeded generator: SplitMix64 on int64 lanes equals the published
-definition on Python integers, values are a pure function of the counter, and
-the synthetic distributions have the stated moments.  CPU only."""
+definition on Python integers, values are a pure function of the counter, the
+synthetic distributions have the stated moments (all on the CPU), and the
+planted prefill inputs are reproducible on the GPU."""
 import numpy as np
+import pytest
 import torch
 
 import workloads as W
@@ -42,3 +44,18 @@ def test_workload_shapes_and_planting():
     assert len(js) == round(0.01 * 256) and bool(torch.all(js[1:] - js[:-1] >= 3))
     c = W.make.make_decode_cache(W.configs.scaled(W.configs.DECODE_BS64_128K, batch=2, L=4096))
     assert c["ic"].shape == (2, 1024, 128) and c["kc_hca"].shape == (2, 32, 128) and c["kw"].shape == (2, 128, 128)
+
+
+@pytest.mark.gpu
+def test_prefill_inputs_are_reproducible_on_the_gpu():
+    # the planted queries are written by indexed assignment; a repeated row index would
+    # make the result depend on which GPU write lands
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    w = W.configs.PREFILL_32K
+    out = []
+    for _ in range(2):
+        raw, qs = W.make.make_raw(w, "cuda"), W.make.make_queries(w, "cuda")
+        W.make.plant_prefill(w, w.layer("csa"), raw, qs, "cuda")
+        out.append((raw["xi"].cpu(), qs["qi"].cpu()))
+    assert torch.equal(out[0][0], out[1][0]) and torch.equal(out[0][1], out[1][1])
