@@ -148,6 +148,13 @@ def _positions(B, T, hi, seed):
     ("bf16", 2, 300, 2000, 64, 4, 64, 0),      # tensor-core scorer, one 64-wide K block
     ("bf16", 2, 300, 1000, 96, 4, 32, 0),      # CUDA-core scorer (width not built for tensor cores)
     ("bf16", 1, 48, 131072, 128, 1, 2048, 0),  # token level (r = 1): 128K raw tokens, k = 2048
+    # decode scorer (one or two query rows per pass): both key widths, both row counts,
+    # passes of 2, 2 and 1 rows, and the fp32 variant
+    ("bf16", 2, 1, 3000, 64, 4, 128, 0),
+    ("bf16", 3, 2, 5000, 64, 4, 256, 0),
+    ("bf16", 4, 2, 6000, 128, 4, 512, 0),
+    ("bf16", 2, 5, 4000, 128, 4, 256, 2),
+    ("f32", 2, 2, 1000, 64, 4, 32, 0),
 ])
 def test_index_flat(S, dtype, B, T, nc, dI, r, k, chunk):
     sc = 1.0 if dtype == "f32" else dI ** -0.5
@@ -175,6 +182,7 @@ def test_index_flat(S, dtype, B, T, nc, dI, r, k, chunk):
     ("bf16", 2, 400, 5000, 128, 128, 8, 256, 4),
     ("bf16", 1, 64, 32768, 128, 128, 64, 2048, 4),
     ("bf16", 1, 48, 131072, 128, 128, 64, 2048, 1),   # token level (r = 1): 1024 blocks of 128 raw tokens
+    ("bf16", 2, 2, 20000, 128, 128, 16, 512, 4),      # decode: stage 1 on the decode scorer
 ])
 def test_index_hisa(S, dtype, B, T, nc, dI, blk, m, k, r):
     sc = 1.0 if dtype == "f32" else dI ** -0.5
