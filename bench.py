@@ -68,15 +68,20 @@ def peaks():
 # --------------------------------------------------------------------------- distributed plumbing
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, timeout_s: float = 300.0):
+    """One process per GPU (RANK / LOCAL_RANK / WORLD_SIZE / MASTER_* from the launcher):
+    NCCL between GPUs; without a GPU (host-side tests of the replica plumbing) gloo."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                             device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=timeout_s)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group("gloo", timeout=timeout)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -88,11 +93,19 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's value (step times are taken as the max over ranks)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(units_per_rank: float, world: int, max_step_ms: float) -> float:
+    """Whole-job rate of `world` independent replicas: every rank's units over the
+    slowest rank's step time."""
+    return world * units_per_rank / (max_step_ms / 1e3)
 
 
 # --------------------------------------------------------------------------- clocks
@@ -767,7 +780,7 @@ def run_ours(args, world, rank, local):
     st, res = bench_prefill(S, w, args.steps, args.warmup, world, flush)
     clocks = clock.stop()
     step_ms = max_over_ranks(res["step_ms"], world)
-    value = world * w.T / (step_ms / 1e3)
+    value = replica_throughput(w.T, world, step_ms)
     attn_ms = res["stage_ms"][2]
     achieved = res["attn_flops"] / (attn_ms / 1e3) / 1e12
     peak = pk["bf16_tflops"]
@@ -821,7 +834,7 @@ def run_ours(args, world, rank, local):
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{pk_src} bf16 burst", "flops_per_launch": res["attn_flops"]},
         "gpu_launches": res["launches"],
-        "e2e": {"value": None if math.isnan(e2e_ms) else world * w.T / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": None if math.isnan(e2e_ms) else replica_throughput(w.T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "clocks": clocks,
