@@ -94,3 +94,12 @@ def test_workspace_sizes(A):
     # of the 148 SMs would hold a query: one sequence splits, 64 do not
     assert A.hyb_attn_fwd_workspace_size(1, 1, 1, 64, 128, 512, 32768, 128, A.HYB_ATTN_DECODE) > 0
     assert A.hyb_attn_fwd_workspace_size(1, 64, 1, 64, 128, 512, 32768, 128, A.HYB_ATTN_DECODE) == 0
+
+
+def test_flat_workspace_budget(A):
+    f = A.hyb_index_topk_workspace_size
+    # the default pass keeps about 512 MiB of fp32 scores, however long the prefill
+    assert f(1, 1, 32768, 8192, 128, 512, A.HYB_INDEX_FLAT) >= 16384 * 8192 * 4
+    assert f(1, 1, 131072, 32768, 128, 2048, A.HYB_INDEX_FLAT) <= (512 << 20) + (1 << 20)
+    # a smaller q_chunk shrinks it (2048 queries x 8192 entries x 4 B = 64 MiB)
+    assert f(1, 1, 32768, 8192, 128, 512, A.HYB_INDEX_FLAT, 0, 0, 2048) <= (64 << 20) + (1 << 20)
