@@ -103,3 +103,18 @@ def test_flat_workspace_budget(A):
     assert f(1, 1, 131072, 32768, 128, 2048, A.HYB_INDEX_FLAT) <= (512 << 20) + (1 << 20)
     # a smaller q_chunk shrinks it (2048 queries x 8192 entries x 4 B = 64 MiB)
     assert f(1, 1, 32768, 8192, 128, 512, A.HYB_INDEX_FLAT, 0, 0, 2048) <= (64 << 20) + (1 << 20)
+
+
+def test_decode_split_rule(A):
+    # split a query's keys into slices only while fewer than half of the 148 SMs would hold
+    # a query: 148 // (2 * queries) slices, at most one per 64 keys; the workspace holds the
+    # fp32 partial outputs and lse of every slice (256-byte aligned)
+    def ws(batch, ns, H=64, D=128):
+        rows = batch * ns * H
+        al = lambda x: (x + 255) // 256 * 256
+        return al(rows * D * 4) + al(rows * 4)
+    f = lambda batch, k, nc: A.hyb_attn_fwd_workspace_size(1, batch, 1, 64, 128, k, nc, 128, A.HYB_ATTN_DECODE)
+    assert f(1, 512, 32768) == ws(1, 10)      # 640 keys: capped at one slice per 64 keys
+    assert f(1, 0, 8192) == ws(1, 64)         # HCA at 1M (8192 entries + 128): 74 capped at 64
+    assert f(37, 512, 32768) == ws(37, 2)     # 148 // 74
+    assert f(38, 512, 32768) == 0             # 148 // 76 = 1: no split
