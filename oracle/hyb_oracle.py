@@ -240,8 +240,8 @@ def key_set(t: int, sel: np.ndarray, kc, vc, kw, vw, ring: int, W: int):
 
 
 def real_kv_positions(t: int, sel: np.ndarray, r: int, W: int) -> np.ndarray:
-    """The "real K/V" reading of CSA attention (SURVEY reading F4; the pages'
-    block-sparse methods attend the real keys and values behind a selection):
+    """The "real K/V" reading of CSA attention (the block-sparse methods the
+    pages compare against attend the real keys and values behind a selection):
     each selected entry j stands for its r raw tokens jr .. jr+r-1, and the key
     set is those tokens together with the window as a set of raw positions (a
     token the window already holds is not repeated), ascending."""
