@@ -248,8 +248,13 @@ def _random_sel(B, T, k, q_pos, r, nc, seed):
     ("f32", 1, 120, 8, 64, 4, 128, 0, 32, 512, "prefill"),
     ("bf16", 2, 150, 64, 128, 2000, 4, 96, 128, 8000, "prefill"),
     ("bf16", 2, 150, 64, 128, 60, 128, 0, 128, 7680, "prefill"),
-    ("bf16", 2, 150, 64, 128, 2000, 4, 96, 128, 8000, "decode"),
-    ("bf16", 3, 2, 64, 128, 60, 128, 0, 128, 7680, "decode"),
+    ("bf16", 2, 150, 64, 128, 2000, 4, 96, 128, 8000, "decode"),   # 300 queries: keys not split
+    ("bf16", 3, 2, 64, 128, 60, 128, 0, 128, 7680, "decode"),      # split-KV: 2 slices
+    ("bf16", 1, 8, 64, 128, 60, 128, 0, 128, 7680, "decode"),      # split-KV: 2 slices; rows at t < 127 see
+                                                                   # no entry: their second slice is empty
+    ("bf16", 2, 4, 64, 128, 2000, 4, 96, 128, 8000, "decode"),     # split-KV: 2 slices
+    ("bf16", 1, 8, 64, 128, 2000, 4, 512, 128, 8000, "decode"),    # split-KV: 5 slices; rows at t = 0..7 see
+                                                                   # at most two entries: slices of masked keys
 ])
 def test_attention(S, dtype, B, T, H, D, nc, r, k, W, L, mode):
     sc = 1.0 if dtype == "f32" else D ** -0.5
@@ -285,7 +290,8 @@ def test_attention(S, dtype, B, T, H, D, nc, r, k, W, L, mode):
     (2, 150, 2000, 4, 96, 128, 8000, "prefill"),
     (2, 150, 2000, 4, 96, 0, 8000, "prefill"),       # no window: the selected tokens alone
     (1, 100, 700, 4, 512, 128, 2800, "prefill"),     # k > visible entries for many rows
-    (2, 150, 2000, 4, 96, 128, 8000, "decode"),      # split-KV schedule
+    (2, 150, 2000, 4, 96, 128, 8000, "decode"),      # 300 queries: keys not split
+    (2, 4, 2000, 4, 96, 128, 8000, "decode"),        # split-KV: 4 slices
 ])
 def test_attention_real_kv(S, B, T, nc, r, k, W, L, mode):
     """The real-K/V reading: selected entries attend their raw tokens (from the ring,
