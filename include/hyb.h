@@ -36,7 +36,10 @@
  *    recorded in a per-device status word, read and cleared by
  *    hyb_get_device_status.  No call traps, asserts or spins without bound.
  *  - Calls are thread-safe and keep no state between calls other than the
- *    per-device status word.
+ *    per-device status word.  One exception: hyb_index_topk_noalloc keeps
+ *    its scores in one fixed device array per GPU, shared by all of its calls
+ *    on that GPU, so two of its calls must never run on one GPU at the same
+ *    time (see its comment).
  */
 #ifndef HYB_H_
 #define HYB_H_
@@ -202,8 +205,10 @@ int hyb_index_topk(int dtype, int batch, int T, int dI,
  * library allocates nothing here either: the scores go to a 16 MiB array that
  * is part of the library's device image, so every GPU that loads libhyb holds
  * those 16 MiB until the process exits.
- *  - The first call on a device (with that device current) looks up the
- *    array's device address; make that first call before any stream capture.
+ *  - Every call looks up the array's device address in the current context
+ *    (a host-side lookup; the address changes if the library's device code is
+ *    loaded again, e.g. after cudaDeviceReset).  The first call on a device
+ *    may load the library's device code; make it before any stream capture.
  *  - All calls on a device share the array.  Calls whose kernels may run at the
  *    same time on that device (different streams without ordering) race on it
  *    and must not be issued.

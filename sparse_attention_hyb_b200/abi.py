@@ -101,6 +101,15 @@ def _ptr(t: Optional[torch.Tensor]):
     return t.data_ptr()
 
 
+def _expect(t: Optional[torch.Tensor], shape, dtype, name: str):
+    """Raises unless `t` has exactly this shape and dtype: the kernels write and
+    read these tensors at the sizes the other arguments imply."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name}: expected {tuple(shape)} {dtype}, got {tuple(t.shape)} {t.dtype}")
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return s.cuda_stream
@@ -181,6 +190,8 @@ def hyb_index_topk_workspace_size(dtype: int, batch: int, T: int, nc: int, dI: i
 def hyb_index_topk(qi, q_pos, ic, nc: int, r: int, k: int, mode: int, reps, block: int, top_m: int,
                    q_chunk: int, idx, ws, stream=None):
     B, T, dI = qi.shape
+    _expect(q_pos, (B, T), torch.int32, "q_pos")
+    _expect(idx, (B, T, k), torch.int32, "idx")
     ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
     st = lib().hyb_index_topk(_dtype_code(qi), B, T, dI, _ptr(qi), _ptr(q_pos), _ptr(ic), nc, ic.shape[1],
                               r, k, mode, _ptr(reps), reps.shape[1] if reps is not None else 0, block,
@@ -191,6 +202,8 @@ def hyb_index_topk(qi, q_pos, ic, nc: int, r: int, k: int, mode: int, reps, bloc
 def hyb_index_topk_noalloc(qi, q_pos, ic, nc: int, r: int, k: int, idx, stream=None):
     """Flat indexer whose scratch is a fixed array inside libhyb (no workspace argument)."""
     B, T, dI = qi.shape
+    _expect(q_pos, (B, T), torch.int32, "q_pos")
+    _expect(idx, (B, T, k), torch.int32, "idx")
     st = lib().hyb_index_topk_noalloc(_dtype_code(qi), B, T, dI, _ptr(qi), _ptr(q_pos), _ptr(ic), nc, ic.shape[1],
                                       r, k, _ptr(idx), _stream(stream))
     _check("hyb_index_topk_noalloc", st)
@@ -204,6 +217,12 @@ def hyb_attn_fwd_workspace_size(dtype: int, batch: int, T: int, H: int, D: int, 
 def hyb_attn_fwd(q, q_pos, kc, vc, nc: int, r: int, idx, k: int, kw, vw, W: int, scale: float, o, lse,
                  mode: int, ws, stream=None):
     B, T, H, D = q.shape
+    _expect(q_pos, (B, T), torch.int32, "q_pos")
+    if idx is not None:
+        _expect(idx, (B, T, k), torch.int32, "idx")
+    _expect(o, (B, T, H, D), q.dtype, "o")
+    if lse is not None:
+        _expect(lse, (B, T, H), torch.float32, "lse")
     ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
     st = lib().hyb_attn_fwd(_dtype_code(q), B, T, H, D, _ptr(q), _ptr(q_pos), _ptr(kc), _ptr(vc), nc,
                             kc.shape[1] if kc is not None else 0, r, _ptr(idx), k, _ptr(kw), _ptr(vw),

@@ -250,6 +250,19 @@ int index_topk_impl(int batch, int T_, int dI, const void* qi, const int* q_pos,
   return HYB_OK;
 }
 
+// Streaming multiprocessors of the current device (148 on B200; also the value
+// used where no device is visible, so that workspace sizes can be queried on a
+// host without a GPU).
+int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return sms;
+}
+
 int attn_splits(int mode, int batch, int T, int n_keys_max) {
   if (mode != HYB_ATTN_DECODE) return 1;
   // a slice is one latency chain of the kernel, and the partial outputs and their
@@ -257,7 +270,7 @@ int attn_splits(int mode, int batch, int T, int n_keys_max) {
   // have a query (batch 64 at 128K: no split, CSA 0.025 ms against 0.035 with two
   // slices and 0.047 with one per key tile), at least 64 keys per split
   const int ctas = batch * T;
-  int ns = 148 / (2 * ctas);
+  int ns = sm_count() / (2 * ctas);
   const int cap = (n_keys_max + 63) / 64;
   if (ns > cap) ns = cap;
   if (ns < 1) ns = 1;
@@ -524,19 +537,14 @@ constexpr size_t kNoAllocScratchBytes = 16u << 20;   // 16 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_noalloc_ptr[kMaxDevices];
-
-// Device address of the scratch array on the current device, looked up once per
-// device (the host-side symbol is not a device address).
+// Device address of the scratch array in the calling thread's current context.
+// The host-side symbol is not a device address, and the address can change when
+// the library's module is loaded again (after cudaDeviceReset, or in another
+// context of the same device), so it is looked up on every call: a host-side
+// table lookup that allocates nothing.
 int noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HYB_ERR_CUDA;
-  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return HYB_ERR_CUDA;
-    g_noalloc_ptr[dev].store(p, std::memory_order_release);
-  }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return HYB_ERR_CUDA;
   *out = p;
   return HYB_OK;
 }
