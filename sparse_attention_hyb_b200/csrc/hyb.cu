@@ -14,6 +14,7 @@
 #include "topk_reg.cuh"
 #include "attn.cuh"
 #include "attn_tc.cuh"
+#include "attn_hm.cuh"
 
 #include <type_traits>
 
@@ -465,10 +466,15 @@ size_t hyb_attn_fwd_workspace_size(int dtype, int batch, int T, int H, int D, in
   return align_up(rows * D * 4) + align_up(rows * 4);
 }
 
-int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const int* q_pos,
-                 const void* kc, const void* vc, int nc, int nc_cap, int r, const int* idx, int k,
-                 const void* kw, const void* vw, int ring, int W, float scale, void* o, float* lse,
-                 int mode, void* ws, size_t ws_bytes, hyb_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int attn_fwd_impl(int dtype, int batch, int T, int H, int D, const void* q, const int* q_pos,
+                  const void* kc, const void* vc, int nc, int nc_cap, int r, const int* idx, int k,
+                  const void* kw, const void* vw, int ring, int W, float scale, void* o, float* lse,
+                  int mode, void* ws, size_t ws_bytes, hyb_stream_t stream, unsigned long long wait_ns,
+                  int drop_arrival) {
   if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
   const bool real_kv = (mode & HYB_ATTN_REAL_KV) != 0;
   mode &= ~HYB_ATTN_REAL_KV;
@@ -495,7 +501,7 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const
     ns = (tiles + per - 1) / per;
   }
   AttnArgs a{q, q_pos, kc, vc, nc, nc_cap, r, idx, k, kw, vw, ring, W, scale, o, lse,
-             nullptr, nullptr, T, H, D, ns, real_kv ? 1 : 0};
+             nullptr, nullptr, T, H, D, ns, real_kv ? 1 : 0, wait_ns, drop_arrival};
   if (ns > 1) {
     const size_t rows = (size_t)batch * T * ns * H;
     const size_t need = align_up(rows * D * 4) + align_up(rows * 4);
@@ -510,13 +516,38 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const
     if (ns > 1) { attn_merge_kernel<float><<<dim3(batch * T, H), 128, 0, s>>>(a); count_launch(); }
   } else {
     if (tc)
-      e = launch_attn_tc(a, batch, s);
+      e = real_kv ? launch_attn_tc(a, batch, s) : launch_attn_hm(a, batch, s);
     else
       e = launch_attn_ffma<bf16>(a, batch, s);
     if (e != cudaSuccess) return HYB_ERR_CUDA;
     if (ns > 1) { attn_merge_kernel<bf16><<<dim3(batch * T, H), 128, 0, s>>>(a); count_launch(); }
   }
   return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const int* q_pos,
+                 const void* kc, const void* vc, int nc, int nc_cap, int r, const int* idx, int k,
+                 const void* kw, const void* vw, int ring, int W, float scale, void* o, float* lse,
+                 int mode, void* ws, size_t ws_bytes, hyb_stream_t stream) {
+  return attn_fwd_impl(dtype, batch, T, H, D, q, q_pos, kc, vc, nc, nc_cap, r, idx, k, kw, vw, ring, W, scale, o,
+                       lse, mode, ws, ws_bytes, stream, sm100::kWaitNs, 0);
+}
+
+int hyb_attn_fwd_wait_test(int dtype, int batch, int T, int H, int D, const void* q, const int* q_pos,
+                           const void* kc, const void* vc, int nc, int nc_cap, int r, const int* idx, int k,
+                           const void* kw, const void* vw, int ring, int W, float scale, void* o, float* lse,
+                           int mode, void* ws, size_t ws_bytes, hyb_stream_t stream, unsigned long long wait_ns,
+                           int drop_arrival) {
+  if (wait_ns == 0 || wait_ns > sm100::kWaitNs) return HYB_ERR_INVALID_ARG;
+  // only the heads-in-M tensor-core kernel has the hook
+  if (dtype != HYB_DTYPE_BF16 || H != attn_hm::kH || D != attn_hm::kD || (mode & HYB_ATTN_REAL_KV))
+    return HYB_ERR_UNSUPPORTED;
+  return attn_fwd_impl(dtype, batch, T, H, D, q, q_pos, kc, vc, nc, nc_cap, r, idx, k, kw, vw, ring, W, scale, o,
+                       lse, mode, ws, ws_bytes, stream, wait_ns, drop_arrival ? 1 : 0);
 }
 
 }  // extern "C"
