@@ -256,6 +256,30 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D,
                  void* o, float* lse, int mode,
                  void* ws, size_t ws_bytes, hyb_stream_t stream);
 
+/*
+ * Test hook for the bounded device waits (no counterpart on the pages: it
+ * exists to exercise the failure path).  Same arguments and results as
+ * hyb_attn_fwd for the tensor-core path it covers (bf16, H = 64, D = 128, not
+ * the real-K/V reading), plus:
+ *  - wait_ns (1 .. 1e9): the limit of every wait inside the attention kernel
+ *    instead of 1 s;
+ *  - drop_arrival != 0: the first CTA withholds one arrival on its first K
+ *    tile, so that its waits expire; that CTA then stops, lets the MMAs it
+ *    issued finish, frees its tensor memory and records HYB_ERR_TIMEOUT in the
+ *    status word (read with hyb_get_device_status).  The outputs of the queries
+ *    that CTA owned are left unspecified; the device and the stream stay usable.
+ * Returns HYB_ERR_INVALID_ARG for wait_ns outside 1 .. 1e9 and
+ * HYB_ERR_UNSUPPORTED for shapes the hook does not cover.
+ */
+int hyb_attn_fwd_wait_test(int dtype, int batch, int T, int H, int D,
+                           const void* q, const int* q_pos,
+                           const void* kc, const void* vc, int nc, int nc_cap, int r,
+                           const int* idx, int k,
+                           const void* kw, const void* vw, int ring, int W, float scale,
+                           void* o, float* lse, int mode,
+                           void* ws, size_t ws_bytes, hyb_stream_t stream,
+                           unsigned long long wait_ns, int drop_arrival);
+
 #ifdef __cplusplus
 }
 #endif

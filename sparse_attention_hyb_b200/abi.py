@@ -49,6 +49,10 @@ SIGNATURES = {
                                 _c_ptr, _c_size, _c_ptr]),
     "hyb_index_topk_noalloc": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_ptr, _c_ptr, _c_ptr, _c_int, _c_int,
                                         _c_int, _c_int, _c_ptr, _c_ptr]),
+    "hyb_attn_fwd_wait_test": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_ptr, _c_ptr, _c_ptr, _c_ptr,
+                                        _c_int, _c_int, _c_int, _c_ptr, _c_int, _c_ptr, _c_ptr, _c_int, _c_int,
+                                        _c_float, _c_ptr, _c_ptr, _c_int, _c_ptr, _c_size, _c_ptr,
+                                        ctypes.c_ulonglong, _c_int]),
     "hyb_attn_fwd_workspace_size": (_c_size, [_c_int] * 9),
     "hyb_attn_fwd": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_ptr, _c_ptr, _c_ptr, _c_ptr,
                               _c_int, _c_int, _c_int, _c_ptr, _c_int, _c_ptr, _c_ptr, _c_int, _c_int,
@@ -229,3 +233,22 @@ def hyb_attn_fwd(q, q_pos, kc, vc, nc: int, r: int, idx, k: int, kw, vw, W: int,
                             kw.shape[1], W, float(scale), _ptr(o), _ptr(lse), mode, _ptr(ws), ws_bytes,
                             _stream(stream))
     _check("hyb_attn_fwd", st)
+
+
+def hyb_attn_fwd_wait_test(q, q_pos, kc, vc, nc: int, r: int, idx, k: int, kw, vw, W: int, scale: float, o, lse,
+                           mode: int, ws, wait_ns: int, drop_arrival: bool, stream=None):
+    """Test hook of the bounded device waits (see include/hyb.h): hyb_attn_fwd with
+    every wait limited to wait_ns, optionally withholding one K-tile arrival."""
+    B, T, H, D = q.shape
+    _expect(q_pos, (B, T), torch.int32, "q_pos")
+    if idx is not None:
+        _expect(idx, (B, T, k), torch.int32, "idx")
+    _expect(o, (B, T, H, D), q.dtype, "o")
+    if lse is not None:
+        _expect(lse, (B, T, H), torch.float32, "lse")
+    ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    st = lib().hyb_attn_fwd_wait_test(_dtype_code(q), B, T, H, D, _ptr(q), _ptr(q_pos), _ptr(kc), _ptr(vc), nc,
+                                      kc.shape[1] if kc is not None else 0, r, _ptr(idx), k, _ptr(kw), _ptr(vw),
+                                      kw.shape[1], W, float(scale), _ptr(o), _ptr(lse), mode, _ptr(ws), ws_bytes,
+                                      _stream(stream), int(wait_ns), int(bool(drop_arrival)))
+    _check("hyb_attn_fwd_wait_test", st)

@@ -23,6 +23,11 @@ struct AttnArgs {
   float* part_o; float* part_lse;  // split-KV partials (nsplit > 1)
   int T, H, D, nsplit;
   int real_kv;  // 1: each selected entry j stands for raw tokens jr .. jr+r-1, read from the ring
+  // Bounded waits of the heads-in-M tensor-core kernel: the limit of every wait, and
+  // a test hook that withholds one K-tile arrival in the first CTA so that the
+  // waits expire (exercises the abort path; 0 in every product call).
+  unsigned long long wait_ns;
+  int test_drop_arrival;
 };
 
 // Key u of query t's list: u < n_comp -> compressed slot u, else window position.
