@@ -180,7 +180,7 @@ def attention_flops(w, ly, q_pos: np.ndarray, n_c: int) -> float:
 
 
 # Sources that define each profiled kernel (its code, helpers and launch).
-KERNEL_SOURCES = {"attention": ["attn_tc.cuh", "attn.cuh", "sm100.cuh", "common.cuh"]}
+KERNEL_SOURCES = {"attention": ["attn_hm.cuh", "attn_tc.cuh", "attn.cuh", "sm100.cuh", "common.cuh"]}
 
 
 def source_hash(kernel: str) -> str:
@@ -287,35 +287,59 @@ def bench_prefill(S, w, steps, warmup, world, flush):
 
 
 def bench_e2e(S, st, steps):
-    """Same step through host buffers: pinned H2D of every input, the three calls,
-    D2H of o and lse, all inside the timed region."""
+    """The same step through host buffers: every step's inputs are copied from
+    pinned host memory and its outputs (o, lse) back, inside the timed region.
+    The copies overlap the compute: two device buffer sets, step i+1's inputs go
+    up on one stream and step i-1's outputs come down on another while step i
+    computes.  Returns (ms per step, H2D bytes per step, D2H bytes per step)."""
     names = ["xk", "xv", "xi", "z"]
     host_raw = {k: st.raw[k].cpu().pin_memory() for k in names}
     host_q = {k: st.qs[k].cpu().pin_memory() for k in ("q", "qi", "q_pos")}
     host_b = st.bias.cpu().pin_memory()
-    out_o = torch.empty(st.o.shape, dtype=st.o.dtype, pin_memory=True)
-    out_l = torch.empty(st.lse.shape, dtype=st.lse.dtype, pin_memory=True)
+    out_o = [torch.empty(st.o.shape, dtype=st.o.dtype, pin_memory=True) for _ in range(2)]
+    out_l = [torch.empty(st.lse.shape, dtype=st.lse.dtype, pin_memory=True) for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in list(host_raw.values()) + list(host_q.values())) \
         + host_b.numel() * 4
-    d2h = out_o.numel() * out_o.element_size() + out_l.numel() * 4
+    d2h = out_o[0].numel() * out_o[0].element_size() + out_l[0].numel() * 4
+    # a second buffer set: inputs, caches, outputs and workspace of its own
+    raw2 = {k: torch.empty_like(v) for k, v in st.raw.items()}
+    qs2 = {k: torch.empty_like(v) for k, v in st.qs.items()}
+    sets = [st, PrefillStep(S, st.w, raw2, qs2, torch.empty_like(st.bias))]
+    up, comp, down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    out_read = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        for k in names:
-            st.raw[k].copy_(host_raw[k], non_blocking=True)
-        for k in host_q:
-            st.qs[k].copy_(host_q[k], non_blocking=True)
-        st.bias.copy_(host_b, non_blocking=True)
-        st.run()
-        out_o.copy_(st.o, non_blocking=True)
-        out_l.copy_(st.lse, non_blocking=True)
+    def step(i):
+        b = i % 2
+        x = sets[b]
+        with torch.cuda.stream(up):
+            up.wait_event(done[b])          # step i-2 no longer reads this set's inputs
+            for k in names:
+                x.raw[k].copy_(host_raw[k], non_blocking=True)
+            for k in host_q:
+                x.qs[k].copy_(host_q[k], non_blocking=True)
+            x.bias.copy_(host_b, non_blocking=True)
+            in_ready[b].record(up)
+        with torch.cuda.stream(comp):
+            comp.wait_event(in_ready[b])
+            comp.wait_event(out_read[b])    # step i-2's outputs have left this set
+            x.run()
+            done[b].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(done[b])
+            out_o[b].copy_(x.o, non_blocking=True)
+            out_l[b].copy_(x.lse, non_blocking=True)
+            out_read[b].record(down)
 
-    one()
+    for i in range(2):
+        step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
+    e0.record(up)
+    for i in range(steps):
+        step(i)
+    e1.record(down)                          # after the last D2H, which follows every copy and call
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
@@ -446,6 +470,32 @@ def graph_times(step, n_seg, steps, warmup, flush):
     return [float(x) for x in np.median(np.array(seg), axis=0)]
 
 
+def selection_iou(a, b) -> float:
+    """Mean over rows of |A & B| / |A | B| for two index sets per row ([R, k] int32,
+    valid entries ascending then -1 padding, as the indexer writes them)."""
+    a, b = a.reshape(-1, a.shape[-1]).long(), b.reshape(-1, b.shape[-1]).long()
+    s, _ = torch.sort(torch.cat([a, b], 1), dim=1)
+    inter = ((s[:, 1:] == s[:, :-1]) & (s[:, 1:] >= 0)).sum(1).float()
+    union = ((a >= 0).sum(1) + (b >= 0).sum(1)).float() - inter
+    return float((inter / union.clamp(min=1)).mean())
+
+
+def planted_recall(idx, qi, ic, planted) -> float:
+    """Fraction of (query, planted entry) pairs with cosine above 0.4 -- the planted
+    construction gives 0.5 -- whose entry the query selected."""
+    if len(planted) == 0:
+        return float("nan")
+    js = torch.as_tensor(planted, device=ic.device).long()
+    q = qi.reshape(-1, qi.shape[-1]).float()
+    kp = ic.reshape(-1, ic.shape[-1])[js].float()
+    cos = (q @ kp.T) / (q.norm(dim=1, keepdim=True) * kp.norm(dim=1)[None, :]).clamp(min=1e-30)
+    r, c = torch.nonzero(cos > 0.4, as_tuple=True)
+    if r.numel() == 0:
+        return float("nan")
+    sel = idx.reshape(-1, idx.shape[-1]).long()
+    return float((sel[r] == js[c][:, None]).any(1).float().mean())
+
+
 def _dense_flops(w, r, n_c, q_pos):
     t = q_pos.astype(np.int64)
     return 4.0 * w.H * w.D * float((np.minimum((t + 1) // r, n_c) + np.minimum(w.W, t + 1)).sum())
@@ -538,11 +588,12 @@ def bench_index_128k(S, steps, warmup, flush):
     A = S.abi
     n_c = w.L // ly.r
     raw = make.make_raw(w, "cuda")
+    qs = make.make_queries(wq, "cuda")
+    planted = make.plant_prefill(wq, ly, raw, qs, "cuda").tolist()
     bias = make.make_bias(w, ly, "cuda")
     kc, vc, ic = S.layer.compress(raw["xk"], raw["xv"], raw["xi"], raw["z"], bias, ly.r, ly.overlap, n_c)
     del raw, kc, vc
     reps = S.layer.block_reps(ic, n_c, ly.block)
-    qs = make.make_queries(wq, "cuda")
     idx = torch.empty(1, wq.T, ly.k, dtype=torch.int32, device="cuda")
     idx2 = torch.empty_like(idx)
     wsf = torch.empty(max(256, A.hyb_index_topk_workspace_size(1, 1, wq.T, n_c, w.dI, ly.k, A.HYB_INDEX_FLAT, 0, 0,
@@ -560,8 +611,67 @@ def bench_index_128k(S, steps, warmup, flush):
         _rec(ev, 2)
 
     flat_ms, hisa_ms = graph_times(step, 2, steps, warmup, flush)
+    step(None)
+    torch.cuda.synchronize()
     return {"workload": "csa_index_128k_last_chunk_bf16", "queries": wq.T, "k": ly.k,
-            "flat_ms": flat_ms, "hisa_ms": hisa_ms, "hisa_speedup": flat_ms / hisa_ms}
+            "flat_ms": flat_ms, "hisa_ms": hisa_ms, "hisa_speedup": flat_ms / hisa_ms,
+            "hisa_vs_flat_iou": selection_iou(idx2, idx),
+            "planted_recall_flat": planted_recall(idx, qs["qi"], ic, planted),
+            "planted_recall_hisa": planted_recall(idx2, qs["qi"], ic, planted),
+            "planted_entries": len(planted)}
+
+
+def bench_prefill_128k(S, steps, warmup, flush, pk):
+    """The whole CSA layer over a 128K-token prefill (all 131072 queries): S1, the
+    flat or the HISA indexer (128-entry blocks, top-64 blocks, query chunk 1024),
+    then attention over the selected top-2048 entries and the window."""
+    w = C.PREFILL_128K
+    ly = w.layer("csa")
+    A = S.abi
+    raw, qs, bias = prefill_inputs(w, "cuda")
+    n_c = w.L // ly.r
+    nb = n_c // ly.block
+    dt = raw["xk"].dtype
+    kc = torch.empty(1, n_c, w.D, dtype=dt, device="cuda")
+    vc, ic = torch.empty_like(kc), torch.empty(1, n_c, w.dI, dtype=dt, device="cuda")
+    reps = torch.empty(1, nb, w.dI, dtype=dt, device="cuda")
+    idx = torch.empty(1, w.T, ly.k, dtype=torch.int32, device="cuda")
+    o, lse = torch.empty_like(qs["q"]), torch.empty(1, w.T, w.H, dtype=torch.float32, device="cuda")
+    wsf = torch.empty(max(256, A.hyb_index_topk_workspace_size(1, 1, w.T, n_c, w.dI, ly.k, A.HYB_INDEX_FLAT, 0, 0, 0)),
+                      dtype=torch.uint8, device="cuda")
+    wsh = torch.empty(max(256, A.hyb_index_topk_workspace_size(1, 1, w.T, n_c, w.dI, ly.k, A.HYB_INDEX_HISA,
+                                                               ly.block, ly.top_m, ly.q_chunk)),
+                      dtype=torch.uint8, device="cuda")
+    scale = 1.0 / math.sqrt(w.D)
+
+    def layer(hisa):
+        def step(ev):
+            _rec(ev, 0)
+            A.hyb_compress(raw["xk"], raw["xv"], raw["xi"], raw["z"], bias, ly.r, ly.overlap, 0, n_c, kc, vc, ic)
+            if hisa:
+                A.hyb_block_reps(ic, ly.block, 0, nb, reps)
+            _rec(ev, 1)
+            if hisa:
+                A.hyb_index_topk(qs["qi"], qs["q_pos"], ic, n_c, ly.r, ly.k, A.HYB_INDEX_HISA, reps, ly.block,
+                                 ly.top_m, ly.q_chunk, idx, wsh)
+            else:
+                A.hyb_index_topk(qs["qi"], qs["q_pos"], ic, n_c, ly.r, ly.k, A.HYB_INDEX_FLAT, None, 0, 0, 0, idx,
+                                 wsf)
+            _rec(ev, 2)
+            A.hyb_attn_fwd(qs["q"], qs["q_pos"], kc, vc, n_c, ly.r, idx, ly.k, raw["xk"], raw["xv"], w.W, scale, o,
+                           lse, A.HYB_ATTN_PREFILL, None)
+            _rec(ev, 3)
+        return step
+
+    out = {"workload": "csa_prefill_128k_bf16", "queries": w.T, "k": ly.k}
+    flops = attention_flops(w, ly, qs["q_pos"][0].cpu().numpy(), n_c)
+    for name, hisa in (("flat", False), ("hisa", True)):
+        c_ms, i_ms, a_ms = graph_times(layer(hisa), 3, max(3, steps // 4), warmup, flush)
+        tot = c_ms + i_ms + a_ms
+        out[f"tokens_per_s_{name}"] = w.T / (tot / 1e3)
+        out[f"stages_ms_{name}"] = {"compress": c_ms, "index_topk": i_ms, "attention": a_ms}
+        out[f"attention_frac_of_bf16_peak_{name}"] = flops / (a_ms / 1e3) / 1e12 / pk["bf16_tflops"]
+    return out
 
 
 def bench_index_128k_tokens(S, steps, warmup, flush):
@@ -594,8 +704,11 @@ def bench_index_128k_tokens(S, steps, warmup, flush):
         _rec(ev, 2)
 
     flat_ms, hisa_ms = graph_times(step, 2, steps, warmup, flush)
+    step(None)
+    torch.cuda.synchronize()
     return {"workload": "token_index_128k_last_chunk_bf16", "queries": wq.T, "k": ly.k, "r": 1,
-            "flat_ms": flat_ms, "hisa_ms": hisa_ms, "hisa_speedup": flat_ms / hisa_ms}
+            "flat_ms": flat_ms, "hisa_ms": hisa_ms, "hisa_speedup": flat_ms / hisa_ms,
+            "hisa_vs_flat_iou": selection_iou(idx2, idx)}
 
 
 def bench_1m(S, steps, warmup, flush, pk):
@@ -682,6 +795,14 @@ def bench_1m(S, steps, warmup, flush, pk):
         _rec(ev, 3)
 
     idx_ms, attn_c_ms, attn_h_ms = graph_times(chunk, 3, steps, warmup, flush)
+    # HISA-vs-flat selection IoU (not timed): the decode row, and the chunk's last 1024 queries
+    torch.cuda.synchronize()
+    iou_dec = selection_iou(idx_d, S.layer.index_topk(qd["qi"], qd["q_pos"], ic_c, ncc, csa.r, csa.k))
+    tail = slice(wc.T - 1024, wc.T)
+    flat_tail = S.layer.index_topk(qc["qi"][:, tail].contiguous(), qc["q_pos"][:, tail].contiguous(), ic_c, ncc, csa.r,
+                                   csa.k)
+    iou_chunk = selection_iou(idx_c[:, tail], flat_tail)
+    del flat_tail
     qp = qc["q_pos"][0].cpu().numpy().astype(np.int64)
     fl_c = 4.0 * wd.H * wd.D * float((np.minimum(np.minimum((qp + 1) // csa.r, ncc), csa.k)
                                        + np.minimum(wd.W, qp + 1)).sum())
@@ -696,29 +817,55 @@ def bench_1m(S, steps, warmup, flush, pk):
         "decode_bs1_ctx1m": {"csa_hisa_ms": dec_csa_ms, "hca_ms": dec_hca_ms,
                              "tokens_per_s_csa_plus_hca": 1.0 / ((dec_csa_ms + dec_hca_ms) / 1e3),
                              "csa_hbm_gbs": dec_bytes_csa / (dec_csa_ms / 1e3) / 1e9,
-                             "hca_hbm_gbs": dec_bytes_hca / (dec_hca_ms / 1e3) / 1e9},
+                             "hca_hbm_gbs": dec_bytes_hca / (dec_hca_ms / 1e3) / 1e9,
+                             "hisa_vs_flat_iou": iou_dec},
         "chunk_prefill_8k_at_1m": {"csa_index_hisa_ms": idx_ms, "csa_attention_ms": attn_c_ms,
                                    "hca_attention_ms": attn_h_ms,
                                    "tokens_per_s_csa": wc.T / ((idx_ms + attn_c_ms) / 1e3),
                                    "tokens_per_s_hca": wc.T / (attn_h_ms / 1e3),
                                    "csa_attention_tflops": fl_c / (attn_c_ms / 1e3) / 1e12,
-                                   "hca_attention_tflops": fl_h / (attn_h_ms / 1e3) / 1e12},
+                                   "hca_attention_tflops": fl_h / (attn_h_ms / 1e3) / 1e12,
+                                   "hisa_vs_flat_iou_last_1024": iou_chunk},
     }
 
 
 # --------------------------------------------------------------------------- CPU oracle
 
 
-def oracle_sample(w, seconds: float):
-    """Times the fp64 oracle on host cores: S1 over the whole sequence, then S2+S3
-    row by row until the budget is spent.  Returns (tokens/s, rows, seconds, cores)."""
+def _oracle_rows_worker(args):
+    """One host core of the CPU baseline: runs the oracle's S2+S3 on its rows (the
+    caches come from the parent through memory-mapped files) until its time budget
+    is spent.  Returns (rows done, seconds spent on them)."""
+    cache_dir, rows, budget, wname = args
+    os.environ["OMP_NUM_THREADS"] = "1"
+    torch.set_num_threads(1)
     import oracle as O
-    try:
-        from threadpoolctl import threadpool_limits
-        limit = threadpool_limits(1)
-    except ImportError:
-        limit = None
-    torch.set_num_threads(os.cpu_count() or 1)
+    w = {c.name: c for c in (C.PREFILL_32K, C.PREFILL_128K)}[wname]
+    ly = w.layer("csa")
+    ld = lambda n: np.load(os.path.join(cache_dir, n + ".npy"), mmap_mode="r")
+    kc, vc, ic, xk, xv, qi64 = (ld(n) for n in ("kc", "vc", "ic", "xk", "xv", "qi"))
+    p = O.LayerParams("csa", ly.r, ly.overlap, w.W, 1.0 / math.sqrt(w.D), w.dtype, k=ly.k)
+    hd = w.H * w.D
+    done, t_rows = 0, 0.0
+    for i in rows:
+        if t_rows >= budget:
+            break
+        q_row = make.to_storage(rng.normal(w.seed, "q", int(i) * hd, hd) * w.x_scale, w.dtype).float().double()
+        t1 = time.perf_counter()
+        O.layer_row(p, q_row.view(w.H, w.D).numpy(), qi64[i], w.q_pos0 + int(i), kc, vc, ic, None, xk, xv,
+                    xk.shape[0])
+        t_rows += time.perf_counter() - t1
+        done += 1
+    return done, t_rows
+
+
+def oracle_sample(w, seconds: float):
+    """Times the fp64 oracle on the host's cores: S1 over the whole sequence in
+    this process, then S2+S3 row by row on every core of the process's affinity
+    mask (one single-threaded worker per core, started with `spawn`) until each
+    worker's budget is spent.  Returns (tokens/s, rows, seconds, cores)."""
+    import multiprocessing as mp
+    import oracle as O
     ly = w.layer("csa")
     raw = make.make_raw(w)
     qi = make.normal_tensor(w.seed, "q_index", (w.batch, w.T, w.dI), w.i_scale, w.dtype)
@@ -731,21 +878,29 @@ def oracle_sample(w, seconds: float):
     kc, vc, ic = O.build_caches(p, f64(raw["xk"][0]), f64(raw["xv"][0]), f64(raw["xi"][0]), f64(raw["z"][0]),
                                 f64(bias))
     t_s1 = time.perf_counter() - t0
-    xk, xv, qi64 = f64(raw["xk"][0]), f64(raw["xv"][0]), f64(qs["qi"][0])
     order = torch.argsort(rng.raw_u64(w.seed, "cpu_rows", 0, w.T)).numpy()
-    done, t_rows = 0, 0.0
-    hd = w.H * w.D
-    while t_rows < seconds and done < w.T:
-        i = int(order[done])
-        q_row = make.to_storage(rng.normal(w.seed, "q", i * hd, hd) * w.x_scale, w.dtype).float().double()
-        t1 = time.perf_counter()
-        O.layer_row(p, q_row.view(w.H, w.D).numpy(), qi64[i], w.q_pos0 + i, kc, vc, ic, None, xk, xv, xk.shape[0])
-        t_rows += time.perf_counter() - t1
-        done += 1
-    if limit is not None:
-        limit.unregister() if hasattr(limit, "unregister") else None
-    per_row = t_rows / done + t_s1 / w.T
-    return 1.0 / per_row, done, t_rows + t_s1, 1
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    cores = max(1, min(cores, 64))
+    with tempfile.TemporaryDirectory() as d:
+        for n, a in (("kc", kc), ("vc", vc), ("ic", ic), ("xk", f64(raw["xk"][0])), ("xv", f64(raw["xv"][0])),
+                     ("qi", f64(qs["qi"][0]))):
+            np.save(os.path.join(d, n + ".npy"), a)
+        jobs = [(d, order[c::cores], seconds, w.name) for c in range(cores)]
+        saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+        os.environ.update({k: "1" for k in saved})   # one BLAS thread per worker (read at the workers' start)
+        try:
+            with mp.get_context("spawn").Pool(cores) as pool:
+                res = pool.map(_oracle_rows_worker, jobs)
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+    done = sum(r[0] for r in res)
+    wall = max(r[1] for r in res)        # the workers run side by side
+    per_row = wall / done + t_s1 / w.T
+    return 1.0 / per_row, done, wall + t_s1, cores
 
 
 # --------------------------------------------------------------------------- arms
@@ -763,7 +918,8 @@ def run_reference(args, world, rank):
         "config": {"workload": w.name, "L": w.L, "T": w.T, "H": w.H, "D": w.D, "dI": w.dI, "r": 4, "k": 512,
                    "W": w.W},
         "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"S1 over all {w.L} tokens + S2/S3 for {rows} seeded rows ({secs:.1f} s)"},
+                         "sample": f"S1 over all {w.L} tokens (1 core) + S2/S3 for {rows} seeded rows on {cores} "
+                                   f"single-threaded workers ({secs:.1f} s)"},
         "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -806,6 +962,8 @@ def run_ours(args, world, rank, local):
         torch.cuda.empty_cache()
         extras["index_128k_last_chunk"] = bench_index_128k(S, args.steps, args.warmup, flush)
         torch.cuda.empty_cache()
+        extras["prefill_128k"] = bench_prefill_128k(S, args.steps, args.warmup, flush, pk)
+        torch.cuda.empty_cache()
         extras["token_index_128k_last_chunk"] = bench_index_128k_tokens(S, args.steps, args.warmup, flush)
         torch.cuda.empty_cache()
         extras.update(bench_1m(S, args.steps, args.warmup, flush, pk))
@@ -816,7 +974,8 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tok_s, rows, secs, cores = oracle_sample(w, args.cpu_seconds)
         cpu = {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"S1 over all {w.L} tokens + S2/S3 for {rows} seeded query rows ({secs:.1f} s, 1 thread)"}
+               "sample": f"S1 over all {w.L} tokens (1 core) + S2/S3 for {rows} seeded query rows on {cores} "
+                         f"single-threaded workers ({secs:.1f} s)"}
     if rank != 0:
         return
     line = {

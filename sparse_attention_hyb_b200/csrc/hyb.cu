@@ -18,7 +18,18 @@
 
 #include <type_traits>
 
+#include <nvtx3/nvToolsExt.h>
+
 using namespace hyb;
+
+namespace {
+// One NVTX range per C-ABI call (visible in Nsight timelines; a no-op when no
+// tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+}  // namespace
 
 namespace {
 
@@ -319,6 +330,7 @@ int hyb_compress(int dtype, int batch, int L, int D, int dI, const void* xk, con
                  const void* xi, const float* logits, const float* bias, int r, int overlap,
                  int j_begin, int j_end, void* kc, void* vc, void* ic, int nc_cap,
                  hyb_stream_t stream) {
+  NvtxRange nvtx_range("hyb_compress");
   if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
   if (batch < 0 || L < 0 || D <= 0 || r < 1 || j_begin < 0 || j_end < j_begin || nc_cap < j_end)
     return HYB_ERR_INVALID_ARG;
@@ -340,6 +352,7 @@ int hyb_compress_pc(int dtype, int batch, int L, int D, int dI, const void* xk, 
                     const float* z_kv, const float* bias_kv, const float* z_i, const float* bias_i, int r,
                     int overlap, int j_begin, int j_end, void* kc, void* vc, void* ic, int nc_cap,
                     hyb_stream_t stream) {
+  NvtxRange nvtx_range("hyb_compress_pc");
   if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
   if (batch < 0 || L < 0 || D <= 0 || r < 1 || j_begin < 0 || j_end < j_begin || nc_cap < j_end)
     return HYB_ERR_INVALID_ARG;
@@ -371,6 +384,7 @@ int hyb_decode_append(int dtype, int batch, int D, int dI, const void* xk_new, c
                       float* zw, int ring, const float* bias_csa, int r_csa, int overlap, void* kc, void* vc,
                       void* ic, int nc_cap, const float* bias_hca, int r_hca, void* kc_hca, void* vc_hca,
                       int nch_cap, int block, void* reps, int nb_cap, hyb_stream_t stream) {
+  NvtxRange nvtx_range("hyb_decode_append");
   if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
   if (batch < 0 || D <= 0 || ring < 1) return HYB_ERR_INVALID_ARG;
   if (batch == 0) return HYB_OK;
@@ -407,6 +421,7 @@ int hyb_decode_append(int dtype, int batch, int D, int dI, const void* xk_new, c
 
 int hyb_block_reps(int dtype, int batch, int dI, const void* ic, int nc_cap, int block, int g_begin,
                    int g_end, void* reps, int nb_cap, hyb_stream_t stream) {
+  NvtxRange nvtx_range("hyb_block_reps");
   if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
   if (batch < 0 || dI <= 0 || block < 1 || g_begin < 0 || g_end < g_begin || g_end > nb_cap ||
       (long long)g_end * block > nc_cap)
@@ -432,6 +447,7 @@ int hyb_index_topk(int dtype, int batch, int T, int dI, const void* qi, const in
                    const void* ic, int nc, int nc_cap, int r, int k, int mode, const void* reps,
                    int nb_cap, int block, int top_m, int q_chunk, int* idx, void* ws,
                    size_t ws_bytes, hyb_stream_t stream) {
+  NvtxRange nvtx_range("hyb_index_topk");
   if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
   if (mode != HYB_INDEX_FLAT && mode != HYB_INDEX_HISA) return HYB_ERR_INVALID_ARG;
   if (batch < 0 || T < 0 || dI <= 0 || nc < 0 || nc_cap < nc || r < 1 || k < 1 || q_chunk < 0)
@@ -533,6 +549,7 @@ int hyb_attn_fwd(int dtype, int batch, int T, int H, int D, const void* q, const
                  const void* kc, const void* vc, int nc, int nc_cap, int r, const int* idx, int k,
                  const void* kw, const void* vw, int ring, int W, float scale, void* o, float* lse,
                  int mode, void* ws, size_t ws_bytes, hyb_stream_t stream) {
+  NvtxRange nvtx_range("hyb_attn_fwd");
   return attn_fwd_impl(dtype, batch, T, H, D, q, q_pos, kc, vc, nc, nc_cap, r, idx, k, kw, vw, ring, W, scale, o,
                        lse, mode, ws, ws_bytes, stream, sm100::kWaitNs, 0);
 }
@@ -542,6 +559,7 @@ int hyb_attn_fwd_wait_test(int dtype, int batch, int T, int H, int D, const void
                            const void* kw, const void* vw, int ring, int W, float scale, void* o, float* lse,
                            int mode, void* ws, size_t ws_bytes, hyb_stream_t stream, unsigned long long wait_ns,
                            int drop_arrival) {
+  NvtxRange nvtx_range("hyb_attn_fwd_wait_test");
   if (wait_ns == 0 || wait_ns > sm100::kWaitNs) return HYB_ERR_INVALID_ARG;
   // only the heads-in-M tensor-core kernel has the hook
   if (dtype != HYB_DTYPE_BF16 || H != attn_hm::kH || D != attn_hm::kD || (mode & HYB_ATTN_REAL_KV))
@@ -584,6 +602,7 @@ int noalloc_scratch(void** out) {
 extern "C" int hyb_index_topk_noalloc(int dtype, int batch, int T, int dI, const void* qi, const int* q_pos,
                                       const void* ic, int nc, int nc_cap, int r, int k, int* idx,
                                       hyb_stream_t stream) {
+  NvtxRange nvtx_range("hyb_index_topk_noalloc");
   if (!dtype_ok(dtype)) return HYB_ERR_UNSUPPORTED;
   if (batch < 0 || T < 0 || dI <= 0 || nc < 0 || nc_cap < nc || r < 1 || k < 1) return HYB_ERR_INVALID_ARG;
   if (batch == 0 || T == 0) return HYB_OK;
