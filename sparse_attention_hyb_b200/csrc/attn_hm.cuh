@@ -56,6 +56,7 @@ namespace attn_hm {
 using attn_tc::Item;
 using attn_tc::KeyList;
 using attn_tc::Maps;
+using attn_tc::div_fast;
 
 constexpr int kH = 64, kD = 128, kTile = 128;
 constexpr int kQSt = 2, kKSt = 3, kVSt = 3, kSBuf = 2, kPBuf = 2, kMSt = 4;
@@ -148,7 +149,8 @@ __device__ __forceinline__ int key_row(const AttnArgs& a, const KeyList& kl, int
   }
   const int u = (tile - kl.comp_tiles) * kTile + rr;
   if (u >= kl.n_win) return -1;
-  return b * a.ring + (kl.w0 + u) % a.ring;
+  const int s = kl.w0_slot + u;   // < 2 ring: u < n_win <= W <= ring
+  return b * a.ring + (s >= a.ring ? s - a.ring : s);
 }
 
 // First global row of a tile whose 128 keys are consecutive valid rows (one TMA box
@@ -160,7 +162,8 @@ __device__ __forceinline__ int tile_box_row(const AttnArgs& a, const KeyList& kl
   }
   const int u0 = (tile - kl.comp_tiles) * kTile;
   if (u0 + kTile > kl.n_win) return -1;
-  const int s0 = (kl.w0 + u0) % a.ring;
+  int s0 = kl.w0_slot + u0;
+  if (s0 >= a.ring) s0 -= a.ring;
   return s0 + kTile <= a.ring ? b * a.ring + s0 : -1;
 }
 
@@ -496,7 +499,9 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         if (!s_have && s_w >= n_items && Gp == Gs) break;
         if (prog) {
           idle = 0;
-        } else if ((++idle & 63u) == 0) {   // no progress: check the abort flag and the time limit
+        } else if (__nanosleep(64), (++idle & 63u) == 0) {
+          // nothing was ready: a short sleep leaves the issue slots of this SMSP to
+          // the softmax warps; every 64 idle rounds, the abort flag and the time limit
           if (abort_flag) break;
           const unsigned long long now = globaltimer();
           if (idle == 64) {
@@ -563,7 +568,7 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
       Item it;
       it.init(a, w, false);
-      const int b = it.kl.row / a.T;
+      const int b = div_fast(it.kl.row, a.T);
       for (int tile = it.tile_beg; tile < it.tile_end && ok; ++tile, ++G) {
         const int st = G % nst;
         const int src = key_row(a, it.kl, b, tile, r_own);   // issued before the slot wait

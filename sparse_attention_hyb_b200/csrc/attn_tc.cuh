@@ -85,14 +85,22 @@ struct Maps {
 
 // Per-query key list: compressed slots [0, n_comp) padded to whole tiles, then
 // the window positions w0 .. w0+n_win-1.
+// x / d and x % d for d > 0, with the common power-of-two divisors (r = 4 or 128,
+// ring lengths, one split) taking a shift instead of a division: every warp of the
+// attention kernels computes this per work item.
+__device__ __forceinline__ int div_fast(int x, int d) { return (d & (d - 1)) == 0 ? x >> (__ffs(d) - 1) : x / d; }
+__device__ __forceinline__ int mod_fast(int x, int d) { return (d & (d - 1)) == 0 ? x & (d - 1) : x % d; }
+
 struct KeyList {
-  int row, t, vis, n_comp, n_win, w0, comp_tiles, tiles;
+  int row, t, vis, n_comp, n_win, w0, w0_slot, comp_tiles, tiles;   // w0_slot = w0 mod ring
   __device__ void init(const AttnArgs& a, int row_, bool real_kv) {
     row = row_;
     t = a.q_pos[row];
-    vis = visible_entries(t, a.r, a.nc);
+    const int v = div_fast(t + 1, a.r);
+    vis = v < a.nc ? v : a.nc;
     n_comp = a.idx ? (real_kv ? a.k * a.r : a.k) : vis;
     w0 = t - a.W + 1 > 0 ? t - a.W + 1 : 0;
+    w0_slot = mod_fast(w0, a.ring);
     n_win = a.W > 0 ? t - w0 + 1 : 0;
     comp_tiles = (n_comp + kTile - 1) / kTile;
     tiles = comp_tiles + (n_win + kTile - 1) / kTile;
@@ -104,10 +112,10 @@ struct Item {
   KeyList kl;
   int split, tile_beg, tile_end;
   __device__ void init(const AttnArgs& a, int w, bool real_kv) {
-    const int row = w / a.nsplit;
-    split = w % a.nsplit;
+    const int row = a.nsplit == 1 ? w : w / a.nsplit;
+    split = a.nsplit == 1 ? 0 : w - row * a.nsplit;
     kl.init(a, row, real_kv);
-    const int per = (kl.tiles + a.nsplit - 1) / a.nsplit;
+    const int per = a.nsplit == 1 ? kl.tiles : (kl.tiles + a.nsplit - 1) / a.nsplit;
     tile_beg = split * per;
     tile_end = min(kl.tiles, tile_beg + per);
     if (tile_beg > tile_end) tile_beg = tile_end;
