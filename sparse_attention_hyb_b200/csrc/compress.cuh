@@ -4,12 +4,19 @@
 // of its position in the window).  CSA windows are 2r long at stride r, HCA
 // windows r long without overlap.
 //
-// HBM-bound streaming pass.  One warp owns one entry: it computes the window's
-// weights once (lanes over window positions) and then pools K, V and the
+// HBM-bound streaming pass.  The pooled sum over a window is defined part by
+// part: parts of kPart consecutive window positions, each summed with fused
+// multiply-adds in ascending position order, then combined in a fixed pairwise
+// grouping (PartSum).  Every path computes exactly this, so the caches are bit-identical
+// whichever kernel wrote them (the decode-step update included).
+// Short windows (CSA, 8 tokens): one warp owns one entry; it computes the
+// window's weights once (lanes over window positions) and pools K, V and the
 // indexer keys with them (lanes over channels, 4 channels per lane, so a warp
-// reads a whole 256-byte bf16 row per load).  Consecutive warps own
-// consecutive entries, so the raw rows shared by two overlapping CSA windows
-// are read twice within a few hundred nanoseconds and the second read hits L2.
+// reads a whole 256-byte bf16 row per load).  Consecutive warps own consecutive
+// entries, so the raw rows shared by two overlapping windows are read twice
+// within a few hundred nanoseconds and the second read hits L2.
+// Long windows (HCA, 128 tokens): one CTA per entry, one warp per part, so that
+// the window's rows are read by several warps at once.
 #pragma once
 #include "common.cuh"
 
@@ -17,6 +24,10 @@ namespace hyb {
 
 constexpr int kCompressWarps = 4;
 constexpr int kMaxSpan = 256;
+constexpr int kPart = 32;                      // window positions per partial sum
+constexpr int kMaxParts = kMaxSpan / kPart;
+constexpr int kPartsMaxC = 256;                // channels of the CTA-per-entry kernel
+constexpr int kPartsEntries = 2048;            // entries below which it is used
 
 // Window weights of one entry into w[0, span): softmax over the in-range tokens
 // (position >= 0) of (logit + bias of the position in the window); z(s) returns
@@ -44,11 +55,68 @@ __device__ __forceinline__ void entry_weights(ZFn z, const float* __restrict__ b
   __syncwarp();
 }
 
-// out[c] = sum_p w[p] * row(start + p)[c] over C channels (4 per lane); row(s)
-// returns the address of token s's row.  One warp.
+__device__ __forceinline__ float4 add4(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+
+// Partial sum of window positions [p0, p1) for the 4 channels at c: fused
+// multiply-adds in ascending position order; positions of weight 0 (before the
+// start of the sequence) are skipped.  NT tensors share the loop (one
+// accumulator each, same arithmetic as NT = 1).
+template <int NT, int UNROLL, typename RowFn>
+__device__ __forceinline__ void pool_part(RowFn row, int c, int start, int p0, int p1, const float* w,
+                                          float4 (&acc)[NT]) {
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll UNROLL
+  for (int p = p0; p < p1; ++p) {
+    const float wp = w[p];
+    if (wp == 0.f) continue;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const float4 v = load4(row(t, start + p) + c);
+      acc[t].x = fmaf(wp, v.x, acc[t].x);
+      acc[t].y = fmaf(wp, v.y, acc[t].y);
+      acc[t].z = fmaf(wp, v.z, acc[t].z);
+      acc[t].w = fmaf(wp, v.w, acc[t].w);
+    }
+  }
+}
+
+// Sum of a window's parts in a fixed pairwise grouping, built part by part like a
+// binary counter: p0 + p1 -> s01, p2 + p3 -> s23, s01 + s23 -> s0123, ...; what is
+// left pending at the end is added from the most recent part upward (with seven
+// parts: s0123 + (s45 + p6)).  Registers only; every path uses this object.
+struct PartSum {
+  float4 l0, l1, l2, l3;   // pending sums of 1, 2, 4 and 8 parts
+  unsigned pend = 0;
+  __device__ __forceinline__ void add(float4 v) {
+    if (!(pend & 1u)) { l0 = v; pend |= 1u; return; }
+    v = add4(l0, v);
+    if (!(pend & 2u)) { l1 = v; pend = (pend & ~1u) | 2u; return; }
+    v = add4(l1, v);
+    if (!(pend & 4u)) { l2 = v; pend = (pend & ~3u) | 4u; return; }
+    v = add4(l2, v);
+    l3 = v;
+    pend = (pend & ~7u) | 8u;
+  }
+  __device__ __forceinline__ float4 total() const {
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+    bool have = false;
+    if (pend & 1u) { r = l0; have = true; }
+    if (pend & 2u) { r = have ? add4(l1, r) : l1; have = true; }
+    if (pend & 4u) { r = have ? add4(l2, r) : l2; have = true; }
+    if (pend & 8u) { r = have ? add4(l3, r) : l3; }
+    return r;
+  }
+};
+
+__host__ __device__ __forceinline__ int n_parts(int span) { return (span + kPart - 1) / kPart; }
+
+// out[c] = sum_p w[p] * row(start + p)[c] over C channels (4 per lane) for a window
+// of one part (span <= kPart): one chain of multiply-adds.  row(s) returns the
+// address of token s's row.  One warp.
 template <typename T, typename RowFn>
-__device__ __forceinline__ void pool_entry(RowFn row, T* __restrict__ out, int C, int start, int span, const float* w,
-                                           int lane) {
+__device__ __forceinline__ void pool_entry_short(RowFn row, T* __restrict__ out, int C, int start, int span,
+                                                 const float* w, int lane) {
   for (int c = lane * 4; c < C; c += 128) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
@@ -65,7 +133,83 @@ __device__ __forceinline__ void pool_entry(RowFn row, T* __restrict__ out, int C
   }
 }
 
+// The same for a window of several parts: each part's chain, then PartSum.  One warp.
+template <typename T, typename RowFn>
+__device__ __forceinline__ void pool_entry_long(RowFn row, T* __restrict__ out, int C, int start, int span,
+                                                const float* w, int lane) {
+  const int np = n_parts(span);
+  auto row1 = [row](int, int s) { return row(s); };
+  for (int c = lane * 4; c < C; c += 128) {
+    PartSum ps;
+#pragma unroll 1
+    for (int q = 0; q < np; ++q) {
+      float4 part[1];
+      pool_part<1, 8>(row1, c, start, q * kPart, min(span, (q + 1) * kPart), w, part);
+      ps.add(part[0]);
+    }
+    store4(out + c, ps.total());
+  }
+}
+
+template <typename T, typename RowFn>
+__device__ __forceinline__ void pool_entry(RowFn row, T* __restrict__ out, int C, int start, int span, const float* w,
+                                           int lane) {
+  if (n_parts(span) == 1) pool_entry_short(row, out, C, start, span, w, lane);
+  else pool_entry_long(row, out, C, start, span, w, lane);
+}
+
+// Long windows: one CTA per entry; warp q computes the window's weights itself and
+// sums part q of the window for K and V (and the indexer keys) in one loop, then
+// the threads combine the parts channel group by channel group.
 template <typename T>
+__global__ void __launch_bounds__(kMaxParts * 32)
+compress_parts_kernel(const T* __restrict__ xk, const T* __restrict__ xv, const T* __restrict__ xi,
+                      const float* __restrict__ logits, const float* __restrict__ bias,
+                      T* __restrict__ kc, T* __restrict__ vc, T* __restrict__ ic,
+                      int L, int D, int dI, int r, int overlap, int j_begin, int nc_cap) {
+  __shared__ float w[kMaxParts][kMaxSpan];
+  __shared__ float4 part[3][kMaxParts][kPartsMaxC / 4];
+  const int b = blockIdx.y, j = j_begin + blockIdx.x;
+  const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int span = overlap ? 2 * r : r, np = n_parts(span);
+  const int start = overlap ? (j - 1) * r : j * r;
+  const float* zb = logits + (size_t)b * L;
+  entry_weights([&](int s) { return zb[s]; }, bias, start, span, w[q], lane);
+  const size_t row0 = (size_t)b * L;
+  const int p0 = q * kPart, p1 = min(span, (q + 1) * kPart);
+  const T* k0 = xk + row0 * D;
+  const T* v0 = xv + row0 * D;
+  for (int c = lane * 4; c < D; c += 128) {
+    float4 acc[2];
+    pool_part<2, 8>([=](int t, int s) { return (t == 0 ? k0 : v0) + (size_t)s * D; }, c, start, p0, p1, w[q], acc);
+    part[0][q][c / 4] = acc[0];
+    part[1][q][c / 4] = acc[1];
+  }
+  if (xi != nullptr)
+    for (int c = lane * 4; c < dI; c += 128) {
+      float4 acc[1];
+      pool_part<1, 8>([=](int, int s) { return xi + (row0 + s) * dI; }, c, start, p0, p1, w[q], acc);
+      part[2][q][c / 4] = acc[0];
+    }
+  __syncthreads();
+  const size_t out0 = (size_t)b * nc_cap + j;
+  for (int g = threadIdx.x; g < D / 4; g += blockDim.x)
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      PartSum ps;
+      for (int i = 0; i < np; ++i) ps.add(part[t][i][g]);
+      store4((t == 0 ? kc : vc) + out0 * D + 4 * g, ps.total());
+    }
+  if (xi != nullptr)
+    for (int g = threadIdx.x; g < dI / 4; g += blockDim.x) {
+      PartSum ps;
+      for (int i = 0; i < np; ++i) ps.add(part[2][i][g]);
+      store4(ic + out0 * dI + 4 * g, ps.total());
+    }
+}
+
+// One warp per entry; LONG: windows of several parts (span > kPart).
+template <typename T, bool LONG>
 __global__ void __launch_bounds__(kCompressWarps * 32)
 compress_kernel(const T* __restrict__ xk, const T* __restrict__ xv, const T* __restrict__ xi,
                 const float* __restrict__ logits, const float* __restrict__ bias,
@@ -83,9 +227,33 @@ compress_kernel(const T* __restrict__ xk, const T* __restrict__ xv, const T* __r
   entry_weights([&](int s) { return zb[s]; }, bias, start, span, w, lane);
   const size_t row0 = (size_t)b * L;
   const size_t out0 = (size_t)b * nc_cap + j;
-  pool_entry([&](int s) { return xk + (row0 + s) * D; }, kc + out0 * D, D, start, span, w, lane);
-  pool_entry([&](int s) { return xv + (row0 + s) * D; }, vc + out0 * D, D, start, span, w, lane);
-  if (xi != nullptr) pool_entry([&](int s) { return xi + (row0 + s) * dI; }, ic + out0 * dI, dI, start, span, w, lane);
+  if constexpr (LONG) {
+    // K and V share each part's loop (twice the loads in flight); each keeps its own
+    // chain, so the arithmetic is that of pool_entry_long
+    const int np = n_parts(span);
+    const T* k0 = xk + row0 * D;
+    const T* v0 = xv + row0 * D;
+    for (int c = lane * 4; c < D; c += 128) {
+      PartSum pk, pv;
+#pragma unroll 1
+      for (int q = 0; q < np; ++q) {
+        float4 acc[2];
+        pool_part<2, 8>([=](int t, int s) { return (t == 0 ? k0 : v0) + (size_t)s * D; }, c, start, q * kPart,
+                        min(span, (q + 1) * kPart), w, acc);
+        pk.add(acc[0]);
+        pv.add(acc[1]);
+      }
+      store4(kc + out0 * D + c, pk.total());
+      store4(vc + out0 * D + c, pv.total());
+    }
+    if (xi != nullptr)
+      pool_entry_long([&](int s) { return xi + (row0 + s) * dI; }, ic + out0 * dI, dI, start, span, w, lane);
+  } else {
+    pool_entry_short([&](int s) { return xk + (row0 + s) * D; }, kc + out0 * D, D, start, span, w, lane);
+    pool_entry_short([&](int s) { return xv + (row0 + s) * D; }, vc + out0 * D, D, start, span, w, lane);
+    if (xi != nullptr)
+      pool_entry_short([&](int s) { return xi + (row0 + s) * dI; }, ic + out0 * dI, dI, start, span, w, lane);
+  }
 }
 
 // S1 with per-channel compression weights: channel c of entry j pools its window
@@ -158,10 +326,21 @@ cudaError_t launch_compress(int batch, int L, int D, int dI, const void* xk, con
                             int nc_cap, cudaStream_t stream) {
   const int n = j_end - j_begin;
   if (n <= 0 || batch <= 0) return cudaSuccess;
+  const int span = overlap ? 2 * r : r;
+  // long windows with too few entries to give every SM several warps (a warp per
+  // entry reads its window part after part): one CTA per entry, one warp per part
+  if (n_parts(span) > 1 && (long long)n * batch < kPartsEntries && D <= kPartsMaxC &&
+      (xi == nullptr || dI <= kPartsMaxC)) {
+    compress_parts_kernel<T><<<dim3(n, batch), n_parts(span) * 32, 0, stream>>>(
+        (const T*)xk, (const T*)xv, (const T*)xi, logits, bias, (T*)kc, (T*)vc, (T*)ic, L, D, dI, r, overlap,
+        j_begin, nc_cap);
+    count_launch();
+    return cudaGetLastError();
+  }
   dim3 grid((n + kCompressWarps - 1) / kCompressWarps, batch);
-  compress_kernel<T><<<grid, kCompressWarps * 32, 0, stream>>>(
-      (const T*)xk, (const T*)xv, (const T*)xi, logits, bias, (T*)kc, (T*)vc, (T*)ic, L, D, dI, r,
-      overlap, j_begin, j_end, nc_cap);
+  auto kern = n_parts(span) > 1 ? compress_kernel<T, true> : compress_kernel<T, false>;
+  kern<<<grid, kCompressWarps * 32, 0, stream>>>((const T*)xk, (const T*)xv, (const T*)xi, logits, bias, (T*)kc,
+                                                 (T*)vc, (T*)ic, L, D, dI, r, overlap, j_begin, j_end, nc_cap);
   count_launch();
   return cudaGetLastError();
 }
