@@ -248,6 +248,30 @@ compress_kernel(const T* __restrict__ xk, const T* __restrict__ xv, const T* __r
     }
     if (xi != nullptr)
       pool_entry_long([&](int s) { return xi + (row0 + s) * dI; }, ic + out0 * dI, dI, start, span, w, lane);
+  } else if (xi != nullptr && dI == D && D <= 128) {
+    // K, V and the indexer keys of the same width share one loop over the window
+    // (one weight read and one skip test per position for the three; each keeps its
+    // own chain of multiply-adds, the arithmetic of pool_entry_short)
+    const int c = lane * 4;
+    if (c < D) {
+      float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, a2 = a0;
+      const T* k0 = xk + row0 * D + c;
+      const T* v0 = xv + row0 * D + c;
+      const T* i0 = xi + row0 * D + c;
+#pragma unroll 4
+      for (int p = 0; p < span; ++p) {
+        const float wp = w[p];
+        if (wp == 0.f) continue;  // token before the start of the sequence
+        const size_t o = (size_t)(start + p) * D;
+        const float4 x0 = load4(k0 + o), x1 = load4(v0 + o), x2 = load4(i0 + o);
+        a0.x = fmaf(wp, x0.x, a0.x); a0.y = fmaf(wp, x0.y, a0.y); a0.z = fmaf(wp, x0.z, a0.z); a0.w = fmaf(wp, x0.w, a0.w);
+        a1.x = fmaf(wp, x1.x, a1.x); a1.y = fmaf(wp, x1.y, a1.y); a1.z = fmaf(wp, x1.z, a1.z); a1.w = fmaf(wp, x1.w, a1.w);
+        a2.x = fmaf(wp, x2.x, a2.x); a2.y = fmaf(wp, x2.y, a2.y); a2.z = fmaf(wp, x2.z, a2.z); a2.w = fmaf(wp, x2.w, a2.w);
+      }
+      store4(kc + out0 * D + c, a0);
+      store4(vc + out0 * D + c, a1);
+      store4(ic + out0 * D + c, a2);
+    }
   } else {
     pool_entry_short([&](int s) { return xk + (row0 + s) * D; }, kc + out0 * D, D, start, span, w, lane);
     pool_entry_short([&](int s) { return xv + (row0 + s) * D; }, vc + out0 * D, D, start, span, w, lane);
