@@ -42,6 +42,7 @@ inline bool dtype_ok(int dtype) { return dtype == HYB_DTYPE_F32 || dtype == HYB_
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA; }
 
 constexpr size_t kSmemTopkMax = 200 * 1024;  // keys staged in shared memory per row
+constexpr int kHisaSlotQueries = 16;            // HISA stage 2 by kept block slot up to this many queries
 constexpr size_t kScoreBudget = 64ull << 20;      // HISA: target bytes of one chunk of block scores + candidates
 constexpr size_t kFlatScoreBudget = 512ull << 20; // flat: target bytes of one chunk of scores
 
@@ -215,7 +216,12 @@ int index_topk_impl(int batch, int T_, int dI, const void* qi, const int* q_pos,
                                                                                nc, block, top_m, p.ldS);
       }
       count_launch();
-      if (hisa_grouped_supported<T>(dI, block, p.nb, qi, ic)) {
+      if ((long long)batch * nq <= kHisaSlotQueries && dI % 4 == 0) {
+        // a few queries (decode): stage 2 in one launch, one CTA per kept block
+        hisa_slot_scores_kernel<T><<<dim3(top_m, nq, batch), 128, dI * 4, stream>>>(
+            (const T*)qi, q_pos, (const T*)ic, blk, SC, ncand, T_, i0, nq, dI, nc_cap, r, nc, block, top_m);
+        count_launch();
+      } else if (hisa_grouped_supported<T>(dI, block, p.nb, qi, ic)) {
         int* list = reinterpret_cast<int*>(ws + p.off_list);
         HgWork* work = reinterpret_cast<HgWork*>(ws + p.off_work);
         int* nwork = reinterpret_cast<int*>(ws + p.off_nwork);

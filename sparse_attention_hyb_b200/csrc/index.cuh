@@ -260,6 +260,50 @@ select_blocks_kernel(const float* __restrict__ SB, const int* __restrict__ q_pos
   if (partial && threadIdx.x == 0) out[full < k1 ? full : k1] = full;
 }
 
+// HISA stage 2 for a few queries (decode): one CTA per (query, kept block slot),
+// one thread per entry of the block, so the whole candidate row is scored in one
+// launch.  Candidate p of a query is entry blk[p / B] * B + p % B (the kept blocks
+// in ascending order, the partial block last); slot 0 also writes the count.
+template <typename T>
+__global__ void __launch_bounds__(128)
+hisa_slot_scores_kernel(const T* __restrict__ qi, const int* __restrict__ q_pos, const T* __restrict__ ic,
+                        const int* __restrict__ blk, float* __restrict__ SC, int* __restrict__ n_cand, int T_, int i0,
+                        int nq, int dI, int nc_cap, int r, int nc, int block, int top_m) {
+  extern __shared__ float qrow[];
+  const int slot = blockIdx.x, m = blockIdx.y, b = blockIdx.z;
+  const size_t row = (size_t)b * T_ + i0 + m;
+  const int v = visible_entries(q_pos[row], r, nc);
+  const int* bl = blk + ((size_t)b * nq + m) * top_m;
+  if (slot == 0 && threadIdx.x == 0) {
+    int n2 = 0;
+    for (int s = 0; s < top_m && bl[s] >= 0; ++s) {
+      const int rem = v - bl[s] * block;
+      n2 += rem < block ? rem : block;
+    }
+    n_cand[(size_t)b * nq + m] = n2;
+  }
+  const int g = bl[slot];
+  if (g < 0) return;
+  const int rem = v - g * block;
+  const int cnt = rem < block ? rem : block;
+  for (int c = threadIdx.x; c < dI; c += blockDim.x) qrow[c] = to_f(qi[row * dI + c]);
+  __syncthreads();
+  float* out = SC + ((size_t)b * nq + m) * ((size_t)top_m * block) + (size_t)slot * block;
+  const T* icb = ic + ((size_t)b * nc_cap + (size_t)g * block) * dI;
+  for (int e = threadIdx.x; e < cnt; e += blockDim.x) {
+    const T* krow = icb + (size_t)e * dI;
+    float acc = 0.f;
+    for (int c = 0; c < dI; c += 4) {
+      const float4 kv = load4(krow + c);
+      acc = fmaf(qrow[c], kv.x, acc);
+      acc = fmaf(qrow[c + 1], kv.y, acc);
+      acc = fmaf(qrow[c + 2], kv.z, acc);
+      acc = fmaf(qrow[c + 3], kv.w, acc);
+    }
+    out[e] = acc;
+  }
+}
+
 // HISA stage 2 scores: candidate p of row (b, i) is entry blocks[p / B] * B + p % B;
 // the valid candidates form a prefix of length n2 (blocks ascending, the
 // partial block last).  One warp per candidate, lanes over channels.

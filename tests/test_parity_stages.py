@@ -183,6 +183,7 @@ def test_index_flat(S, dtype, B, T, nc, dI, r, k, chunk):
     ("bf16", 1, 64, 32768, 128, 128, 64, 2048, 4),
     ("bf16", 1, 48, 131072, 128, 128, 64, 2048, 1),   # token level (r = 1): 1024 blocks of 128 raw tokens
     ("bf16", 2, 2, 20000, 128, 128, 16, 512, 4),      # decode: stage 1 on the decode scorer
+    ("f32", 2, 3, 3000, 32, 16, 6, 40, 4),            # a few queries: stage 2 by kept-block slot, B = 16
 ])
 def test_index_hisa(S, dtype, B, T, nc, dI, blk, m, k, r):
     sc = 1.0 if dtype == "f32" else dI ** -0.5
