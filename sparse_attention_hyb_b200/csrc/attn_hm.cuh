@@ -499,9 +499,9 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         if (!s_have && s_w >= n_items && Gp == Gs) break;
         if (prog) {
           idle = 0;
-        } else if (__nanosleep(64), (++idle & 63u) == 0) {
-          // nothing was ready: a short sleep leaves the issue slots of this SMSP to
-          // the softmax warps; every 64 idle rounds, the abort flag and the time limit
+        } else if ((++idle & 63u) == 0) {
+          // nothing was ready (the issuer spins: measured faster than sleeping between
+          // rounds); every 64 idle rounds, the abort flag and the time limit
           if (abort_flag) break;
           const unsigned long long now = globaltimer();
           if (idle == 64) {
