@@ -28,8 +28,11 @@
 //               compressed range) is one 2-D TMA box per 64-column half.  K
 //               producers also publish the tile's validity mask (ballot).
 // Ring depths: 2 Q, 3 K, 3 V tiles in shared memory (224 KB); in tensor memory
-// two S buffers (free as soon as the softmax has loaded them), two P buffers and
-// one O accumulator (512 columns).
+// three S buffers and one O accumulator (512 columns).  P_G (bf16 pairs) is
+// written over the first half of S_G's buffer once both softmax warps of a
+// quadrant have loaded it (their exchange of the row maximum orders the two), so
+// the softmax never waits for an O update before storing P; S_{G+3} waits for
+// the O update of tile G, which frees the buffer.
 //
 // Softmax: the running maximum m (base-2 units) only moves when a tile exceeds it
 // by more than 8, and then O in tensor memory and the row sum are rescaled after
@@ -59,17 +62,16 @@ using attn_tc::Maps;
 using attn_tc::div_fast;
 
 constexpr int kH = 64, kD = 128, kTile = 128;
-constexpr int kQSt = 2, kKSt = 3, kVSt = 3, kSBuf = 2, kPBuf = 2, kMSt = 4;
+constexpr int kQSt = 2, kKSt = 3, kVSt = 3, kSBuf = 3, kMSt = 4;
 constexpr int kSmxWarps = 8, kMmaWarp = 8, kQWarp = 9, kKWarp0 = 10, kVWarp0 = 14;
 constexpr int kThreads = 18 * 32;
 constexpr int kQBytes = kH * kD * 2;      // 16 KB: two 64-column halves of 64 rows x 128 B
 constexpr int kKVBytes = kTile * kD * 2;  // 32 KB: two 64-column halves of 128 rows x 128 B
 constexpr int kSmem = kQSt * kQBytes + (kKSt + kVSt) * kKVBytes + 1024;
 static_assert(kMSt > kKSt, "the mask ring must not hold back the K producers");
-constexpr uint32_t kSCols = 128;                  // one S buffer: 128 fp32 columns (0 .. 255)
-constexpr uint32_t kPCol = kSBuf * kSCols;        // P buffers: 64 columns of bf16 pairs each (256 .. 383)
-constexpr uint32_t kPCols = 64;
-constexpr uint32_t kOCol = kPCol + kPBuf * kPCols; // O accumulator: columns 384 .. 511
+constexpr uint32_t kSCols = 128;              // one S buffer: 128 fp32 columns (three: 0 .. 383);
+                                              // P over its first 64 columns
+constexpr uint32_t kOCol = kSBuf * kSCols;    // O accumulator: columns 384 .. 511
 constexpr float kRescaleThreshold = 8.f;
 
 // ------------------------------------------------------------ tensor-memory access
@@ -177,7 +179,7 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
   uint8_t* sV = sK + kKSt * kKVBytes;
 
   __shared__ uint64_t q_full[kQSt], q_empty[kQSt], k_full[kKSt], k_empty[kKSt], v_full[kVSt], v_empty[kVSt];
-  __shared__ uint64_t s_full[kSBuf], s_read[kSBuf], p_full[kPBuf], o_bar[2], o_free, m_full[kMSt], m_empty[kMSt];
+  __shared__ uint64_t s_full[kSBuf], p_full[kSBuf], o_bar[kSBuf], o_free, m_full[kMSt], m_empty[kMSt];
   __shared__ uint64_t mma_done;
   __shared__ __align__(16) uint32_t mask[kMSt][4];
   __shared__ uint64_t xbar[4][2], lbar[4];     // softmax pair exchanges (per lane quadrant)
@@ -191,9 +193,8 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     for (int s = 0; s < kQSt; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
     for (int s = 0; s < kKSt; ++s) { mbar_init(&k_full[s], 128); mbar_init(&k_empty[s], 1); }
     for (int s = 0; s < kVSt; ++s) { mbar_init(&v_full[s], 128); mbar_init(&v_empty[s], 1); }
-    for (int s = 0; s < kSBuf; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_read[s], kSmxWarps); }
-    for (int s = 0; s < kPBuf; ++s) mbar_init(&p_full[s], kSmxWarps);
-    for (int s = 0; s < 2; ++s) mbar_init(&o_bar[s], 1);
+    for (int s = 0; s < kSBuf; ++s) { mbar_init(&s_full[s], 1); mbar_init(&p_full[s], kSmxWarps); }
+    for (int s = 0; s < kSBuf; ++s) mbar_init(&o_bar[s], 1);
     mbar_init(&o_free, kSmxWarps);
     for (int s = 0; s < kMSt; ++s) { mbar_init(&m_full[s], 4); mbar_init(&m_empty[s], kSmxWarps); }
     for (int s = 0; s < 4; ++s) { mbar_init(&xbar[s][0], 2); mbar_init(&xbar[s][1], 2); mbar_init(&lbar[s], 2); }
@@ -218,15 +219,12 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
     const int h = q4 * 16 + r16;              // head row
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const float c2 = a.scale * 1.4426950408889634f;   // scale * log2(e)
-    uint32_t G = 0, cons = 0, n_ep = 0;       // tiles processed; O updates observed; epilogues done
+    uint32_t G = 0, n_ep = 0;                 // tiles processed; epilogues done
     bool ok = true;
-    // observe O updates 0 .. need-1 complete; `ok` stays warp-uniform (the
+    // waits until the O update of tile g completed; `ok` stays warp-uniform (the
     // tensor-memory accesses that follow are warp-collective)
-    auto consume_until = [&](uint32_t need) {
-      while (cons < need && ok) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&o_bar[cons & 1], (cons >> 1) & 1u, &abort_flag, lim));
-        ++cons;
-      }
+    auto wait_o = [&](uint32_t g) {
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_bar[g % kSBuf], full_par(g, kSBuf), &abort_flag, lim));
     };
     // one value per head row shared with the partner warp through `slot`, ordered by
     // the pair's barrier `bar` (phase `par`); returns the partner's value
@@ -264,7 +262,7 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
       float m_use = 0.f, l = 0.f;   // running maximum (base-2 units) and this thread's part of the row sum
       bool m_set = false;
       for (int tile = it.tile_beg; tile < it.tile_end && ok; ++tile, ++G) {
-        const int sb = G % kSBuf, pb_ = G % kPBuf, ms = G % kMSt;
+        const int sb = G % kSBuf, ms = G % kMSt;
         const bool last = tile + 1 == it.tile_end;
         ok = mbar_wait(&m_full[ms], full_par(G, kMSt), &abort_flag, lim) && ok;
         const uint4 mw = *reinterpret_cast<const uint4*>(mask[ms]);
@@ -279,9 +277,7 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         ld16x2_x16(lane_addr + sb * kSCols + 64 * hw, sa);
         ld16x2_x16(lane_addr + sb * kSCols + 64 * hw + 32, sbv);
         tmem_wait_ld();
-        fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_read[sb]);   // the S buffer may take a later tile now
+        fence_before_sync();   // the partner's P store into this buffer follows the exchange
         // masked keys score -inf (probability exactly 0); a tile whose keys are all
         // valid (full tiles: the common case) skips the per-key tests
         float x[32];
@@ -311,6 +307,7 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
         mt = fmaxf(mt, exchange(mt, red[G & 1][hw][q4], red[G & 1][hw ^ 1][q4], &xbar[q4][G & 1], (G >> 1) & 1u)) * c2;
         if (!ok) break;
+        fence_after_sync();
         float alpha = 1.f;
         bool resc = false;
         if (!m_set) {
@@ -320,11 +317,11 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           m_use = mt;
           resc = true;
         }
-        // before P_G is written, the O update of tile G-2 must be observed: it read the
-        // same P buffer, and no o_bar barrier may run two phases ahead of this warp;
-        // G-1 when rescaling O
+        // rescaling O waits for the O update of tile G-1.  A wait on o_bar for tile g
+        // cannot alias another phase: the update of g-3 completed before S_g was
+        // issued, and the update of g+3 needs P_{g+3}, which this warp writes later
         const bool wresc = __any_sync(0xffffffffu, resc);
-        consume_until(wresc ? G : (G >= 2 ? G - 1 : 0));
+        if (wresc) wait_o(G - 1);
         if (wresc && ok) {
           fence_after_sync();
 #pragma unroll 1
@@ -359,15 +356,15 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         }
         l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
         if (!ok) break;
-        st16x2_x8(lane_addr + kPCol + pb_ * kPCols + 32 * hw, pa);
-        st16x2_x8(lane_addr + kPCol + pb_ * kPCols + 32 * hw + 16, pb);
+        st16x2_x8(lane_addr + sb * kSCols + 32 * hw, pa);
+        st16x2_x8(lane_addr + sb * kSCols + 32 * hw + 16, pb);
         tmem_wait_st();
         fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[pb_]);
+        if (lane == 0) mbar_arrive(&p_full[sb]);
         if (!last) continue;
         // ---- epilogue of the item: every O update of it complete, then o = O / l
-        consume_until(G + 1);
+        wait_o(G);
         if (!ok) break;
         fence_after_sync();
         float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
@@ -421,8 +418,8 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
       const uint64_t dq0 = desc_kmajor_sw128(smem_u32(sQ)), dk0 = desc_kmajor_sw128(smem_u32(sK));
       const uint64_t dv0 = desc_mnmajor_sw128(smem_u32(sV), kKVBytes / 2);
       // Two in-order streams scheduled by readiness: S of later tiles as K tiles and
-      // S buffers free up, O updates as probabilities arrive; neither waits for the
-      // other.
+      // S buffers free up (the O update that read a buffer's P completed), O updates
+      // as probabilities arrive; neither waits for the other.
       Item s_it, p_it;
       int s_w = blockIdx.x, p_w = blockIdx.x, s_tile = 0, p_tile = 0;
       bool s_have = false, p_have = false;
@@ -438,12 +435,12 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           }
           if (s_w < n_items) { s_have = true; s_tile = s_it.tile_beg; }
         }
-        // ---- S stream: S_G = Q . K_G^T into buffer G % 2 (free once the softmax loaded S_{G-2})
+        // ---- S stream: S_G = Q . K_G^T into buffer G % 3 (free once the O update of G-3 completed)
         if (s_have) {
           const int sb = Gs % kSBuf, ks = Gs % kKSt, qs = nq % kQSt;
           const bool first = s_tile == s_it.tile_beg;
           if ((!first || mbar_test_wait(&q_full[qs], full_par(nq, kQSt))) &&
-              mbar_test_wait(&s_read[sb], empty_par(Gs, kSBuf)) && mbar_test_wait(&k_full[ks], full_par(Gs, kKSt))) {
+              mbar_test_wait(&o_bar[sb], empty_par(Gs, kSBuf)) && mbar_test_wait(&k_full[ks], full_par(Gs, kKSt))) {
             fence_after_sync();
             const uint64_t da = dq0 + (uint64_t)((qs * kQBytes) >> 4), db = dk0 + (uint64_t)((ks * kKVBytes) >> 4);
             const uint32_t d = tmem + sb * kSCols;
@@ -475,18 +472,18 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
             p_have = true;
             p_tile = p_it.tile_beg;
           }
-          const int pb = Gp % kPBuf, vs = Gp % kVSt;
+          const int pb = Gp % kSBuf, vs = Gp % kVSt;
           const bool first = p_tile == p_it.tile_beg;
           if ((!first || items_done == 0 || mbar_test_wait(&o_free, (items_done - 1) & 1u)) &&
-              mbar_test_wait(&p_full[pb], full_par(Gp, kPBuf)) && mbar_test_wait(&v_full[vs], full_par(Gp, kVSt))) {
+              mbar_test_wait(&p_full[pb], full_par(Gp, kSBuf)) && mbar_test_wait(&v_full[vs], full_par(Gp, kVSt))) {
             fence_after_sync();
             const uint64_t db = dv0 + (uint64_t)((vs * kKVBytes) >> 4);
-            const uint32_t ta = tmem + kPCol + pb * kPCols;
+            const uint32_t ta = tmem + pb * kSCols;
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk)
               mma_f16_ts(tmem + kOCol, ta + kk * 8, db + ((kk * 2048) >> 4), idO, (first && kk == 0) ? 0u : 1u);
             mma_commit(&v_empty[vs]);
-            mma_commit(&o_bar[Gp & 1]);
+            mma_commit(&o_bar[pb]);
             ++Gp;
             if (++p_tile == p_it.tile_end) {
               ++items_done;
