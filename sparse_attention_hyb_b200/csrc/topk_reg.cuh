@@ -6,13 +6,15 @@
 // keys (blocked layout: thread t owns positions [t*EPT, (t+1)*EPT)).  A 12-bit
 // radix pass (4096-bin shared histogram) finds the bin that holds the k-th
 // largest key.  The keys of that bin are gathered into shared memory (normally
-// a few hundred at most) and one warp runs three more radix passes over them
-// alone (8, 8 and 4 bits), which give the exact k-th key K* and how many keys
-// equal to it are taken; rows where more keys share the bin run a 12-bit and
-// an 8-bit pass over the registers.
-// Because the layout is blocked, the ordered output needs a single block-wide
-// exclusive scan of per-thread (greater-than, equal-to) counts; every thread
-// then writes its selected positions in ascending order.
+// a few hundred at most) and one warp resolves them alone: up to 32 by counting,
+// for each, the candidates above and equal to it; more by radix passes (8, 8 and
+// 4 bits); either gives the exact k-th key K* and how many keys equal to it are
+// taken.  Rows where more keys share the bin run a 12-bit and an 8-bit pass
+// over the registers.
+// Because the layout is blocked, a thread's selected elements form one bit mask
+// (keys above K*, plus the first equal ones); the ordered output needs a single
+// block-wide exclusive scan of per-thread (greater-than, equal-to) counts, and
+// every thread then writes the positions of its mask's bits in ascending order.
 #pragma once
 #include "common.cuh"
 #include "topk.cuh"
@@ -122,51 +124,69 @@ __device__ __forceinline__ void find_digit(RegSelSmem<THREADS>& sh, int shift) {
   __syncthreads();
 }
 
-// One warp finds the remaining 20 bits of the k-th key among the n boundary-bin
-// candidates in shared memory: three radix passes (bits 19..12, 11..4, 3..0) over a
-// 256-bin histogram of its own, warp-synchronous only; leaves prefix / remaining
-// as find_digit does.
+// One warp finds the k-th key among the n boundary-bin candidates in shared
+// memory (every candidate shares the `done_bits` high bits already fixed in
+// sh.prefix; sh.remaining is the rank sought among them).  Up to 32 candidates:
+// each lane counts the candidates above and equal to its own; more: radix
+// passes of up to 8 bits over a 256-bin histogram of the warp's own.  Leaves
+// prefix = K* and remaining = how many keys equal to K* are taken.
 template <int THREADS>
-__device__ __forceinline__ void resolve_candidates_warp(RegSelSmem<THREADS>& sh, uint32_t n) {
+__device__ __forceinline__ void resolve_candidates_warp(RegSelSmem<THREADS>& sh, uint32_t n, int done_bits) {
   const int lane = threadIdx.x & 31;
-  uint32_t prefix = sh.prefix, rem = sh.remaining, mask = 0xFFF00000u;
-  uint32_t* h = sh.hist;
+  uint32_t prefix = sh.prefix, rem = sh.remaining;
+  if (n <= 32) {
+    const uint32_t mine = (uint32_t)lane < n ? sh.cand_key[lane] : 0u;
+    uint32_t gt = 0, eq = 0;
+    for (uint32_t j = 0; j < n; ++j) {
+      const uint32_t kj = __shfl_sync(0xffffffffu, mine, j);
+      gt += kj > mine ? 1u : 0u;
+      eq += kj == mine ? 1u : 0u;
+    }
+    const bool hit = (uint32_t)lane < n && gt < rem && rem <= gt + eq;
+    const int src = __ffs(__ballot_sync(0xffffffffu, hit)) - 1;
+    prefix = __shfl_sync(0xffffffffu, mine, src);
+    rem -= __shfl_sync(0xffffffffu, gt, src);
+  } else {
+    uint32_t mask = done_bits ? ~0u << (32 - done_bits) : 0u;
+    uint32_t* h = sh.hist;
 #pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 12 : (pass == 1 ? 4 : 0);
-    const uint32_t dmask = pass == 2 ? 0xFu : 0xFFu;
-    for (int i = lane; i < 256; i += 32) h[i] = 0u;
-    __syncwarp();
-    for (uint32_t c = lane; c < n; c += 32) {
-      const uint32_t kc = sh.cand_key[c];
-      if ((kc & mask) == prefix) atomicAdd(&h[(kc >> shift) & dmask], 1u);
-    }
-    __syncwarp();
-    uint32_t v[8], tot = 0;   // lane l owns digits 8l .. 8l+7
-#pragma unroll
-    for (int e = 0; e < 8; ++e) { v[e] = h[lane * 8 + e]; tot += v[e]; }
-    uint32_t incl = tot;      // keys in this lane's digits and above
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t u = __shfl_down_sync(0xffffffffu, incl, o);
-      if (lane + o < 32) incl += u;
-    }
-    uint32_t above = incl - tot, d = 0, nrem = 0;
-    const bool mine = above < rem && rem <= above + tot;
-    if (mine) {
-#pragma unroll
-      for (int e = 7; e >= 0; --e) {
-        if (above + v[e] >= rem) { d = lane * 8 + e; nrem = rem - above; break; }
-        above += v[e];
+    for (int low = 32 - done_bits; low > 0;) {
+      const int nb = low < 8 ? low : 8, shift = low - nb;
+      const uint32_t dmask = (1u << nb) - 1u;
+      for (int i = lane; i < 256; i += 32) h[i] = 0u;
+      __syncwarp();
+      for (uint32_t c = lane; c < n; c += 32) {
+        const uint32_t kc = sh.cand_key[c];
+        if ((kc & mask) == prefix) atomicAdd(&h[(kc >> shift) & dmask], 1u);
       }
+      __syncwarp();
+      uint32_t v[8], tot = 0;   // lane l owns digits 8l .. 8l+7
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { v[e] = h[lane * 8 + e]; tot += v[e]; }
+      uint32_t incl = tot;      // keys in this lane's digits and above
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += u;
+      }
+      uint32_t above = incl - tot, d = 0, nrem = 0;
+      const bool mine = above < rem && rem <= above + tot;
+      if (mine) {
+#pragma unroll
+        for (int e = 7; e >= 0; --e) {
+          if (above + v[e] >= rem) { d = lane * 8 + e; nrem = rem - above; break; }
+          above += v[e];
+        }
+      }
+      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+      d = __shfl_sync(0xffffffffu, d, src);
+      nrem = __shfl_sync(0xffffffffu, nrem, src);
+      prefix |= d << shift;
+      rem = nrem;
+      mask |= dmask << shift;
+      low = shift;
+      __syncwarp();
     }
-    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-    d = __shfl_sync(0xffffffffu, d, src);
-    nrem = __shfl_sync(0xffffffffu, nrem, src);
-    prefix |= d << shift;
-    rem = nrem;
-    mask |= dmask << shift;
-    __syncwarp();
   }
   if (lane == 0) { sh.prefix = prefix; sh.remaining = rem; }
 }
@@ -237,7 +257,7 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
     for (int e = 0; e < EPT; ++e)
       if (e < cnt && (key[e] >> 20) == (prefix0 >> 20)) sh.cand_key[slot++] = key[e];
     __syncthreads();
-    if (tid < 32) resolve_candidates_warp<THREADS>(sh, n_cand);
+    if (tid < 32) resolve_candidates_warp<THREADS>(sh, n_cand, 12);
     __syncthreads();
   } else {
     // many keys share the first digit: a 12-bit and an 8-bit pass over the registers
@@ -258,29 +278,33 @@ __device__ void select_row_reg(const float* __restrict__ scores, int n, int k, i
     find_digit<THREADS, kLastBins>(sh, 0);
   }
   const uint32_t kth = sh.prefix, need = sh.remaining;
-  // ---- ordered output
-  uint32_t gt = 0, eq = 0;
+  // ---- ordered output: bit e of gtm / eqm marks element e above / equal to K*
+  static_assert(EPT <= 32, "one mask word per thread");
+  uint32_t gtm = 0, eqm = 0;
 #pragma unroll
-  for (int e = 0; e < EPT; ++e)
-    if (e < cnt) { gt += key[e] > kth; eq += key[e] == kth; }
+  for (int e = 0; e < EPT; ++e) {
+    if (e < cnt) {
+      gtm |= (key[e] > kth ? 1u : 0u) << e;
+      eqm |= (key[e] == kth ? 1u : 0u) << e;
+    }
+  }
+  const uint32_t n_gt = __popc(gtm), n_eq = __popc(eqm);
   uint32_t total;
-  const uint32_t before = block_exclusive_scan<THREADS>((gt << 16) | eq, sh, total);
-  uint32_t gt_run = before >> 16, eq_run = before & 0xFFFFu;
+  const uint32_t before = block_exclusive_scan<THREADS>((n_gt << 16) | n_eq, sh, total);
+  const uint32_t gt_before = before >> 16, eq_before = before & 0xFFFFu;
+  // the equal keys taken are the first `need` in position order
+  const uint32_t take = eq_before >= need ? 0u : min(need - eq_before, n_eq);
+  while ((uint32_t)__popc(eqm) > take) eqm &= ~(0x80000000u >> __clz(eqm));   // drop the highest
+  uint32_t sel = gtm | eqm;
   // selected positions in ascending order: staged in shared memory when k fits,
   // then stored by consecutive threads
   const bool staged = k <= kSelOut;
   int* dst = staged ? sh.outbuf : out;
-#pragma unroll
-  for (int e = 0; e < EPT; ++e) {
-    if (e >= cnt) break;
-    const uint32_t kv = key[e];
-    if (kv > kth) {
-      dst[gt_run + (eq_run < need ? eq_run : need)] = map(base + e);
-      ++gt_run;
-    } else if (kv == kth) {
-      if (eq_run < need) dst[gt_run + eq_run] = map(base + e);
-      ++eq_run;
-    }
+  uint32_t slot = gt_before + min(eq_before, need);
+  while (sel) {
+    const int e = __ffs(sel) - 1;
+    dst[slot++] = map(base + e);
+    sel &= sel - 1;
   }
   if (staged) {
     __syncthreads();
