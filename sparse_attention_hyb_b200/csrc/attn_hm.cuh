@@ -439,8 +439,11 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         if (s_have) {
           const int sb = Gs % kSBuf, ks = Gs % kKSt, qs = nq % kQSt;
           const bool first = s_tile == s_it.tile_beg;
-          if ((!first || mbar_test_wait(&q_full[qs], full_par(nq, kQSt))) &&
-              mbar_test_wait(&o_bar[sb], empty_par(Gs, kSBuf)) && mbar_test_wait(&k_full[ks], full_par(Gs, kKSt))) {
+          // the three tests are issued together (not short-circuited), so their latencies overlap
+          const bool c1 = !first || mbar_test_wait(&q_full[qs], full_par(nq, kQSt));
+          const bool c2 = mbar_test_wait(&o_bar[sb], empty_par(Gs, kSBuf));
+          const bool c3 = mbar_test_wait(&k_full[ks], full_par(Gs, kKSt));
+          if (c1 & c2 & c3) {
             fence_after_sync();
             const uint64_t da = dq0 + (uint64_t)((qs * kQBytes) >> 4), db = dk0 + (uint64_t)((ks * kKVBytes) >> 4);
             const uint32_t d = tmem + sb * kSCols;
@@ -474,8 +477,10 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           }
           const int pb = Gp % kSBuf, vs = Gp % kVSt;
           const bool first = p_tile == p_it.tile_beg;
-          if ((!first || items_done == 0 || mbar_test_wait(&o_free, (items_done - 1) & 1u)) &&
-              mbar_test_wait(&p_full[pb], full_par(Gp, kSBuf)) && mbar_test_wait(&v_full[vs], full_par(Gp, kVSt))) {
+          const bool c1 = !first || items_done == 0 || mbar_test_wait(&o_free, (items_done - 1) & 1u);
+          const bool c2 = mbar_test_wait(&p_full[pb], full_par(Gp, kSBuf));
+          const bool c3 = mbar_test_wait(&v_full[vs], full_par(Gp, kVSt));
+          if (c1 & c2 & c3) {
             fence_after_sync();
             const uint64_t db = dv0 + (uint64_t)((vs * kKVBytes) >> 4);
             const uint32_t ta = tmem + pb * kSCols;

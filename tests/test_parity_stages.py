@@ -177,6 +177,34 @@ def test_index_flat(S, dtype, B, T, nc, dI, r, k, chunk):
     assert np.mean(ious) >= 0.999
 
 
+@pytest.mark.parametrize("T,nc,dI,k,lo,hi", [
+    (40, 6000, 32, 512, -3, 4),     # scores: small integers, hundreds of keys per value
+    (40, 9000, 8, 2048, -1, 2),     # a few dozen distinct values, thousands of keys each
+    (24, 20000, 16, 1024, -2, 3),   # rows of up to 20000 keys (the 1024-thread select)
+])
+def test_index_flat_exact_ties(S, T, nc, dI, k, lo, hi):
+    """Integer-valued fp32 keys and queries make every score exact (sums of small
+    integer products) and put whole groups of keys at the k-th score: the selection
+    must equal the oracle's rule exactly, ties going to the lower entry.  Query row 4
+    (which sees every entry) is all zeros, so all of its scores tie."""
+    B = 2
+    ic = (rng.randint_below(11, "tie_ic", 0, B * nc * dI, hi - lo) + lo).view(B, nc, dI).to(torch.float32)
+    qi = (rng.randint_below(11, "tie_qi", 0, B * T * dI, hi - lo) + lo).view(B, T, dI).to(torch.float32)
+    qi[:, 4] = 0.0
+    q_pos = _positions(B, T, 4 * nc + 40, 6)
+    idx = S.layer.index_topk(qi.to(dev), q_pos.to(dev), ic.to(dev), nc, 4, k)
+    torch.cuda.synchronize()
+    idx = idx.cpu().numpy()
+    for b in range(B):
+        ic64, qi64 = to64(ic[b]), to64(qi[b])
+        for i in range(T):
+            n = O.visible_entries(int(q_pos[b, i]), 4, nc)
+            ids = np.arange(n)
+            want = O.select_topk(O.index_scores(qi64[i], ic64, ids), ids, k)
+            want = np.concatenate([np.sort(want[want >= 0]), want[want < 0]])   # ascending, then -1
+            assert np.array_equal(idx[b, i], want), f"b{b} row {i} (n = {n})"
+
+
 @pytest.mark.parametrize("dtype,B,T,nc,dI,blk,m,k,r", [
     ("f32", 1, 200, 300, 32, 16, 4, 20, 4),
     ("bf16", 2, 400, 5000, 128, 128, 8, 256, 4),
