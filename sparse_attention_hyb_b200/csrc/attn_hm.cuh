@@ -39,7 +39,9 @@
 // the previous O update completed; otherwise probabilities are taken against the
 // stale maximum (they stay below 2^8).  Masked keys (indexer padding, entries
 // outside the visible range, window positions past the query) get probability 0
-// and their rows are zero-filled without a global read.
+// and their rows are zero-filled without a global read.  A query's epilogue
+// (o = O / l, lse) runs one tile late, inside the next query's first tile just
+// before its P store, so the softmax does not wait for the query's last O update.
 //
 // A work item is a query, or in split-KV decode a tile-aligned slice of its keys
 // whose partial (o, lse) attn_merge combines.  Every wait is bounded (AttnArgs::
@@ -235,6 +237,59 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar, par, &abort_flag, lim)) && ok;
       return slot_other[r16];
     };
+    // ---- epilogue of an item: its last O update complete, then o = O / l (deferred by one tile)
+    bool pend = false, e_final = true;
+    size_t e_prow = 0;
+    float e_m = 0.f, e_l = 0.f;
+    uint32_t e_G = 0;
+    auto epilogue = [&]() {
+      pend = false;
+      const float l = e_l, m_use = e_m;
+      const size_t prow = e_prow;
+      const bool final_out = e_final;
+      wait_o(e_G);
+      if (!ok) return;
+      fence_after_sync();
+      float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      lt += exchange(lt, redl[hw][q4], redl[hw ^ 1][q4], &lbar[q4], n_ep & 1u);
+      ++n_ep;
+      if (!ok) return;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      uint32_t ov[2][16];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) ld16x2_x16(lane_addr + kOCol + 64 * hw + 32 * c, ov[c]);
+      tmem_wait_ld();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free);   // the accumulator may be overwritten by the next item
+      if (hw == 0 && hi == 0) {
+        const float lse = lt > 0.f ? m_use * 0.6931471805599453f + logf(lt) : -INFINITY;
+        if (final_out) { if (a.lse) a.lse[prow + h] = lse; }
+        else a.part_lse[prow + h] = lse;
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int d0 = 64 * hw + 32 * c + 16 * hi;
+        if (final_out) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            __nv_bfloat162 x2 = __floats2bfloat162_rn(__uint_as_float(ov[c][2 * i]) * inv,
+                                                      __uint_as_float(ov[c][2 * i + 1]) * inv);
+            pk[i] = *reinterpret_cast<uint32_t*>(&x2);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<bf16*>(a.o) + (prow + h) * kD + d0);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else {
+          float4* dst = reinterpret_cast<float4*>(a.part_o + (prow + h) * kD + d0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_float4(__uint_as_float(ov[c][4 * i]) * inv, __uint_as_float(ov[c][4 * i + 1]) * inv,
+                                 __uint_as_float(ov[c][4 * i + 2]) * inv, __uint_as_float(ov[c][4 * i + 3]) * inv);
+        }
+      }
+    };
     for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
       Item it;
       it.init(a, w, false);
@@ -356,58 +411,30 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
         }
         l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
         if (!ok) break;
+        // the previous item's epilogue runs here, before this tile's P store: its last O
+        // update had most of a tile's time to complete, and reading O frees the accumulator
+        // before the new item's first O update can be issued
+        if (pend) {
+          epilogue();
+          if (!ok) break;
+        }
         st16x2_x8(lane_addr + sb * kSCols + 32 * hw, pa);
         st16x2_x8(lane_addr + sb * kSCols + 32 * hw + 16, pb);
         tmem_wait_st();
         fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[sb]);
-        if (!last) continue;
-        // ---- epilogue of the item: every O update of it complete, then o = O / l
-        wait_o(G);
-        if (!ok) break;
-        fence_after_sync();
-        float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
-        lt += exchange(lt, redl[hw][q4], redl[hw ^ 1][q4], &lbar[q4], n_ep & 1u);
-        ++n_ep;
-        if (!ok) break;
-        const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        uint32_t ov[2][16];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) ld16x2_x16(lane_addr + kOCol + 64 * hw + 32 * c, ov[c]);
-        tmem_wait_ld();
-        fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&o_free);   // the accumulator may be overwritten by the next item
-        if (hw == 0 && hi == 0) {
-          const float lse = lt > 0.f ? m_use * 0.6931471805599453f + logf(lt) : -INFINITY;
-          if (final_out) { if (a.lse) a.lse[prow + h] = lse; }
-          else a.part_lse[prow + h] = lse;
-        }
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int d0 = 64 * hw + 32 * c + 16 * hi;
-          if (final_out) {
-            uint32_t pk[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              __nv_bfloat162 x2 = __floats2bfloat162_rn(__uint_as_float(ov[c][2 * i]) * inv,
-                                                        __uint_as_float(ov[c][2 * i + 1]) * inv);
-              pk[i] = *reinterpret_cast<uint32_t*>(&x2);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<bf16*>(a.o) + (prow + h) * kD + d0);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          } else {
-            float4* dst = reinterpret_cast<float4*>(a.part_o + (prow + h) * kD + d0);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_float4(__uint_as_float(ov[c][4 * i]) * inv, __uint_as_float(ov[c][4 * i + 1]) * inv,
-                                   __uint_as_float(ov[c][4 * i + 2]) * inv, __uint_as_float(ov[c][4 * i + 3]) * inv);
-          }
+        if (last) {
+          pend = true;
+          e_prow = prow;
+          e_final = final_out;
+          e_m = m_use;
+          e_l = l;
+          e_G = G;
         }
       }
     }
+    if (pend && ok) epilogue();
   } else if (warp == kMmaWarp) {
     // ======================================================== MMA issuer
     if (lane == 0) {
