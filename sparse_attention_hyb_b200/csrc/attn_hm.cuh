@@ -462,37 +462,8 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
           }
           if (s_w < n_items) { s_have = true; s_tile = s_it.tile_beg; }
         }
-        // ---- S stream: S_G = Q . K_G^T into buffer G % 3 (free once the O update of G-3 completed)
-        if (s_have) {
-          const int sb = Gs % kSBuf, ks = Gs % kKSt, qs = nq % kQSt;
-          const bool first = s_tile == s_it.tile_beg;
-          // the three tests are issued together (not short-circuited), so their latencies overlap
-          const bool c1 = !first || mbar_test_wait(&q_full[qs], full_par(nq, kQSt));
-          const bool c2 = mbar_test_wait(&o_bar[sb], empty_par(Gs, kSBuf));
-          const bool c3 = mbar_test_wait(&k_full[ks], full_par(Gs, kKSt));
-          if (c1 & c2 & c3) {
-            fence_after_sync();
-            const uint64_t da = dq0 + (uint64_t)((qs * kQBytes) >> 4), db = dk0 + (uint64_t)((ks * kKVBytes) >> 4);
-            const uint32_t d = tmem + sb * kSCols;
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_f16_ss(d, da + ((c * (kQBytes / 2) + kk * 32) >> 4), db + ((c * (kKVBytes / 2) + kk * 32) >> 4),
-                           idS, (c | kk) != 0);
-            mma_commit(&k_empty[ks]);
-            mma_commit(&s_full[sb]);
-            ++Gs;
-            if (++s_tile == s_it.tile_end) {
-              mma_commit(&q_empty[qs]);
-              ++nq;
-              s_have = false;
-              s_w += gridDim.x;
-            }
-            prog = true;
-          }
-        }
-        // ---- O stream: O += P_G . V_G once the softmax wrote P_G
+        // ---- O stream first: O += P_G . V_G once the softmax wrote P_G (an O update frees
+        // the S/P buffer that S of tile G+3 waits for)
         if (Gp < Gs) {
           if (!p_have) {
             for (; p_w < n_items; p_w += gridDim.x) {
@@ -521,6 +492,36 @@ attn_hm_kernel(const __grid_constant__ Maps maps, AttnArgs a, int n_items) {
               ++items_done;
               p_have = false;
               p_w += gridDim.x;
+            }
+            prog = true;
+          }
+        }
+        // ---- S stream: S_G = Q . K_G^T into buffer G % 3 (free once the O update of G-3 completed)
+        if (s_have) {
+          const int sb = Gs % kSBuf, ks = Gs % kKSt, qs = nq % kQSt;
+          const bool first = s_tile == s_it.tile_beg;
+          // the three tests are issued together (not short-circuited), so their latencies overlap
+          const bool c1 = !first || mbar_test_wait(&q_full[qs], full_par(nq, kQSt));
+          const bool c2 = mbar_test_wait(&o_bar[sb], empty_par(Gs, kSBuf));
+          const bool c3 = mbar_test_wait(&k_full[ks], full_par(Gs, kKSt));
+          if (c1 & c2 & c3) {
+            fence_after_sync();
+            const uint64_t da = dq0 + (uint64_t)((qs * kQBytes) >> 4), db = dk0 + (uint64_t)((ks * kKVBytes) >> 4);
+            const uint32_t d = tmem + sb * kSCols;
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_f16_ss(d, da + ((c * (kQBytes / 2) + kk * 32) >> 4), db + ((c * (kKVBytes / 2) + kk * 32) >> 4),
+                           idS, (c | kk) != 0);
+            mma_commit(&k_empty[ks]);
+            mma_commit(&s_full[sb]);
+            ++Gs;
+            if (++s_tile == s_it.tile_end) {
+              mma_commit(&q_empty[qs]);
+              ++nq;
+              s_have = false;
+              s_w += gridDim.x;
             }
             prog = true;
           }
