@@ -118,3 +118,32 @@ def test_decode_split_rule(A):
     assert f(1, 0, 8192) == ws(1, 64)         # HCA at 1M (8192 entries + 128): 74 capped at 64
     assert f(37, 512, 32768) == ws(37, 2)     # 148 // 74
     assert f(38, 512, 32768) == 0             # 148 // 76 = 1: no split
+
+
+def test_binding_checks_shapes_and_types_before_the_call(A):
+    """The Python binding refuses output and position tensors whose shape or type
+    differs from what the other arguments imply (the kernels would write past them);
+    the checks run before the library is called, so host tensors suffice here."""
+    import torch
+    B, T, dI, nc, k, H, D = 2, 3, 16, 40, 8, 64, 128
+    qi, ic = torch.zeros(B, T, dI), torch.zeros(B, nc, dI)
+    q_pos = torch.zeros(B, T, dtype=torch.int32)
+    idx = torch.zeros(B, T, k, dtype=torch.int32)
+    bad_idx = [torch.zeros(B, T, k - 1, dtype=torch.int32), torch.zeros(B, T, k, dtype=torch.int64), None]
+    for bi in bad_idx:
+        with pytest.raises(ValueError, match="idx"):
+            A.hyb_index_topk(qi, q_pos, ic, nc, 4, k, 0, None, 0, 0, 0, bi, None)
+        with pytest.raises(ValueError, match="idx"):
+            A.hyb_index_topk_noalloc(qi, q_pos, ic, nc, 4, k, bi)
+    with pytest.raises(ValueError, match="q_pos"):
+        A.hyb_index_topk(qi, q_pos.long(), ic, nc, 4, k, 0, None, 0, 0, 0, idx, None)
+    q = torch.zeros(B, T, H, D, dtype=torch.bfloat16)
+    kw = torch.zeros(B, 128, D, dtype=torch.bfloat16)
+    o, lse = torch.zeros_like(q), torch.zeros(B, T, H)
+    args = (q, q_pos, None, None, 0, 4, idx, k, kw, kw, 128, 0.1)
+    with pytest.raises(ValueError, match="o:"):
+        A.hyb_attn_fwd(*args, o.float(), lse, 0, None)
+    with pytest.raises(ValueError, match="lse"):
+        A.hyb_attn_fwd(*args, o, lse[:, :, :-1], 0, None)
+    with pytest.raises(ValueError, match="idx"):
+        A.hyb_attn_fwd(q, q_pos, None, None, 0, 4, bad_idx[0], k, kw, kw, 128, 0.1, o, lse, 0, None)
